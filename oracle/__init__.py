@@ -1,0 +1,155 @@
+"""CPU oracle for the W4A16 group-128 linear layer (TEST INFRASTRUCTURE ONLY).
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline
+leg may import this package.  The CUDA library never calls it, links it or
+shares code with it.
+
+The arithmetic lives in ``w4a16_oracle.c`` (plain C, FP32 with separate
+roundings, sequential over k).  This wrapper only builds it with gcc and
+marshals numpy arrays; BF16 travels as uint16 bit patterns.
+
+Every oracle function is pinned by ``tests/test_oracle_pins.py``; the pins
+are in turn shown to reject deliberately broken copies of the C source by
+``tests/test_oracle_mutants.py``.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+SOURCE = os.path.join(HERE, "w4a16_oracle.c")
+LIBRARY = os.path.join(HERE, "libw4a16_oracle.so")
+CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+          "-std=c11", "-Wall", "-Wextra", "-Werror"]
+
+
+def compile_source(src: str, out: str) -> str:
+    tmp = out + f".tmp{os.getpid()}"
+    subprocess.run(["gcc", *CFLAGS, src, "-o", tmp], check=True)
+    os.replace(tmp, out)
+    return out
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc if the shared object is missing or stale."""
+    stale = (not os.path.exists(LIBRARY)) or os.path.getmtime(LIBRARY) < os.path.getmtime(SOURCE)
+    if force or stale:
+        compile_source(SOURCE, LIBRARY)
+    return LIBRARY
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a, dtype=dtype)
+    return a, a.ctypes.data_as(ctypes.c_void_p)
+
+
+class Oracle:
+    """ctypes view of one build of ``w4a16_oracle.c``."""
+
+    def __init__(self, path: str):
+        lib = ctypes.CDLL(path)
+        p, i64 = ctypes.c_void_p, ctypes.c_int64
+        for name in ("w4a16_oracle_matmul", "w4a16_oracle_matmul_f32"):
+            fn = getattr(lib, name)
+            fn.argtypes = [p, p, p, p, p, i64, i64, i64]
+            fn.restype = ctypes.c_int
+        lib.w4a16_oracle_unpack.argtypes = [p, p, i64, i64]
+        lib.w4a16_oracle_unpack.restype = ctypes.c_int
+        lib.w4a16_oracle_round_bf16.argtypes = [p, p, i64]
+        lib.w4a16_oracle_round_bf16.restype = None
+        lib.w4a16_oracle_threads.argtypes = []
+        lib.w4a16_oracle_threads.restype = ctypes.c_int
+        lib.w4a16_oracle_set_threads.argtypes = [ctypes.c_int]
+        lib.w4a16_oracle_set_threads.restype = None
+        self.lib = lib
+        self.path = path
+
+    @staticmethod
+    def _inputs(x, wq, scales, biases):
+        x, px = _c(x, np.uint16)
+        wq, pw = _c(wq, np.uint32)
+        s, ps = _c(scales, np.uint16)
+        b, pb = _c(biases, np.uint16)
+        M, K = x.shape
+        N = wq.shape[0]
+        G = K // 128 if K % 128 == 0 else -1
+        if wq.shape != (N, K // 8) or s.shape != (N, G) or b.shape != (N, G):
+            raise ValueError("shape mismatch between x, wq, scales and biases")
+        return (x, wq, s, b), (px, pw, ps, pb), M, N, K
+
+    def matmul(self, x, wq, scales, biases) -> np.ndarray:
+        """y [M,N] BF16 bits = x . dequant(wq)^T (FP32 sequential accumulation)."""
+        keep, ptrs, M, N, K = self._inputs(x, wq, scales, biases)
+        y = np.empty((M, N), dtype=np.uint16)
+        if self.lib.w4a16_oracle_matmul(*ptrs, y.ctypes.data_as(ctypes.c_void_p), M, N, K):
+            raise ValueError("oracle rejected its arguments")
+        return y
+
+    def matmul_f32(self, x, wq, scales, biases) -> np.ndarray:
+        """The FP32 accumulator before the final BF16 rounding."""
+        keep, ptrs, M, N, K = self._inputs(x, wq, scales, biases)
+        acc = np.empty((M, N), dtype=np.float32)
+        if self.lib.w4a16_oracle_matmul_f32(*ptrs, acc.ctypes.data_as(ctypes.c_void_p), M, N, K):
+            raise ValueError("oracle rejected its arguments")
+        return acc
+
+    def unpack(self, wq, K: int) -> np.ndarray:
+        wq, pw = _c(wq, np.uint32)
+        N = wq.shape[0]
+        q = np.empty((N, K), dtype=np.uint8)
+        if self.lib.w4a16_oracle_unpack(pw, q.ctypes.data_as(ctypes.c_void_p), N, K):
+            raise ValueError("oracle rejected its arguments")
+        return q
+
+    def round_bf16(self, a) -> np.ndarray:
+        a, pa = _c(a, np.float32)
+        out = np.empty(a.shape, dtype=np.uint16)
+        self.lib.w4a16_oracle_round_bf16(pa, out.ctypes.data_as(ctypes.c_void_p), a.size)
+        return out
+
+    def threads(self) -> int:
+        return self.lib.w4a16_oracle_threads()
+
+    def set_threads(self, n: int) -> None:
+        self.lib.w4a16_oracle_set_threads(int(n))
+
+
+_lock = threading.Lock()
+_default = None
+
+
+def default() -> Oracle:
+    global _default
+    with _lock:
+        if _default is None:
+            _default = Oracle(build())
+    return _default
+
+
+def matmul(x, wq, scales, biases):
+    return default().matmul(x, wq, scales, biases)
+
+
+def matmul_f32(x, wq, scales, biases):
+    return default().matmul_f32(x, wq, scales, biases)
+
+
+def unpack(wq, K):
+    return default().unpack(wq, K)
+
+
+def round_bf16(a):
+    return default().round_bf16(a)
+
+
+def threads():
+    return default().threads()
+
+
+def set_threads(n):
+    default().set_threads(n)

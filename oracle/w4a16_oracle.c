@@ -1,0 +1,159 @@
+/*
+ * Plain CPU oracle for the W4A16 group-128 linear layer.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing in the library's compute path may call,
+ * link or include this file; only the tests, the smoke check and the
+ * benchmark's CPU-baseline leg do.  It shares no code with the CUDA library.
+ *
+ * What it computes (tiny-llm, "Week 2 Day 6: SIMD-Matrix Prefill": the
+ * introduction fixes 4-bit weights, group size 128, BF16 activations, BF16
+ * quantisation parameters, BF16 output and FP32 accumulators; Task 3 fixes one
+ * scale and one bias per 128 reduction values):
+ *
+ *   1. unpack   q[n,k] = (wq[n*(K/8) + k/8] >> (4*(k%8))) & 15
+ *   2. dequant  w[n,k] = float(s[n,k/128]) * float(q[n,k]) + float(b[n,k/128])
+ *               (two FP32 roundings: the product, then the sum)
+ *   3. dot      acc = 0; for k = 0..K-1: acc = acc + float(x[m,k]) * w[n,k]
+ *               (FP32, product and sum rounded separately, k ascending)
+ *   4. store    y[m,n] = bf16_round_to_nearest_even(acc)
+ *
+ * This is the plain definition; it must be compiled without contraction of
+ * a*b+c into fused multiply-adds (-ffp-contract=off) and without fast-math.
+ * Outputs are independent, so they may be computed by several threads; the
+ * arithmetic of each output is the sequence above regardless.
+ *
+ * BF16 values are passed as uint16_t bit patterns.
+ */
+#include <stdint.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#if defined(__FAST_MATH__)
+#error "the oracle must not be built with fast-math"
+#endif
+
+static float bf16_to_f32(uint16_t h)
+{
+    uint32_t u = (uint32_t)h << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+static uint16_t f32_to_bf16_rne(float f)
+{
+    uint32_t u;
+    memcpy(&u, &f, sizeof u);
+    if ((u & 0x7f800000u) == 0x7f800000u) {          /* inf or nan */
+        if (u & 0x007fffffu)
+            return (uint16_t)((u >> 16) | 0x0040u);  /* quiet nan */
+        return (uint16_t)(u >> 16);
+    }
+    /* add half an ulp of bf16, plus one more when the kept lsb is odd: ties go to even */
+    u += 0x7fffu + ((u >> 16) & 1u);
+    return (uint16_t)(u >> 16);
+}
+
+static unsigned unpack_code(const uint32_t *wq, int64_t K, int64_t n, int64_t k)
+{
+    uint32_t word = wq[n * (K / 8) + k / 8];
+    return (unsigned)((word >> (4 * (k % 8))) & 15u);
+}
+
+static float dot_fp32(const uint16_t *x, const uint32_t *wq, const uint16_t *s,
+                      const uint16_t *b, int64_t K, int64_t m, int64_t n)
+{
+    const int64_t G = K / 128;
+    float acc = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        const float sc = bf16_to_f32(s[n * G + k / 128]);
+        const float bi = bf16_to_f32(b[n * G + k / 128]);
+        const float q = (float)unpack_code(wq, K, n, k);
+        const float sq = sc * q;
+        const float w = sq + bi;
+        const float xv = bf16_to_f32(x[m * K + k]);
+        const float p = xv * w;
+        acc = acc + p;
+    }
+    return acc;
+}
+
+/* Status: 0 ok, 1 bad argument (null pointer, negative size, K % 128 != 0). */
+static int check(const void *x, const void *wq, const void *s, const void *b,
+                 const void *y, int64_t M, int64_t N, int64_t K)
+{
+    if (M < 0 || N < 0 || K < 0 || K % 128 != 0)
+        return 1;
+    if (M > 0 && N > 0 && (!x || !wq || !s || !b || !y))
+        return 1;
+    return 0;
+}
+
+/* y[M,N] bf16 bits = x[M,K] . dequant(wq)^T, steps 1-4 above. */
+int w4a16_oracle_matmul(const uint16_t *x, const uint32_t *wq, const uint16_t *s,
+                        const uint16_t *b, uint16_t *y, int64_t M, int64_t N,
+                        int64_t K)
+{
+    if (check(x, wq, s, b, y, M, N, K))
+        return 1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            y[m * N + n] = f32_to_bf16_rne(dot_fp32(x, wq, s, b, K, m, n));
+    return 0;
+}
+
+/* Same as above but stops before step 4: the FP32 accumulator itself. */
+int w4a16_oracle_matmul_f32(const uint16_t *x, const uint32_t *wq, const uint16_t *s,
+                            const uint16_t *b, float *acc, int64_t M, int64_t N,
+                            int64_t K)
+{
+    if (check(x, wq, s, b, acc, M, N, K))
+        return 1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            acc[m * N + n] = dot_fp32(x, wq, s, b, K, m, n);
+    return 0;
+}
+
+/* Step 1 alone: q[N,K] codes as bytes. */
+int w4a16_oracle_unpack(const uint32_t *wq, uint8_t *q, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % 8 != 0 || (N > 0 && K > 0 && (!wq || !q)))
+        return 1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (uint8_t)unpack_code(wq, K, n, k);
+    return 0;
+}
+
+/* Step 4 alone, for the rounding pins: float32 -> bf16 bits. */
+void w4a16_oracle_round_bf16(const float *a, uint16_t *out, int64_t count)
+{
+    for (int64_t i = 0; i < count; ++i)
+        out[i] = f32_to_bf16_rne(a[i]);
+}
+
+/* Number of OpenMP threads a parallel region would use (1 without OpenMP). */
+int w4a16_oracle_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* Cap the threads later parallel regions use (no effect without OpenMP). */
+void w4a16_oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    if (n > 0)
+        omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

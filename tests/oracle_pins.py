@@ -1,0 +1,269 @@
+"""Pins that tie the CPU oracle to facts other than its own code.
+
+Each function takes an ``oracle.Oracle`` (the real build, or a deliberately
+broken copy in ``test_oracle_mutants.py``) and raises AssertionError when the
+oracle disagrees with:
+
+* hand-derived values stored under ``tests/golden/`` (unpacking of hand-built
+  words, BF16 round-to-nearest-even ties, FP32 accumulation corner cases);
+* closed forms (identity weights reproduce x; one-hot activations read single
+  codes; all-ones activations give per-column sums of the dequantised weights);
+* exact integer arithmetic (integer-valued inputs whose FP32 sums are exact);
+* exact rational arithmetic on tiny random problems, within the FP32 error
+  bound of recursive summation.
+
+Expected values never come from the oracle or the CUDA library.
+"""
+from __future__ import annotations
+
+import os
+from fractions import Fraction
+
+import numpy as np
+
+import w4a16_synth as synth
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _golden_lines(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line
+
+
+def _expand(field):
+    out = []
+    for tok in field.split():
+        if "*" in tok:
+            v, r = tok.split("*")
+            out += [int(v, 0)] * int(r)
+        else:
+            out.append(int(tok, 0))
+    return out
+
+
+def _bits_to_fraction(bits: int) -> Fraction:
+    """Exact value of a BF16 bit pattern (finite only)."""
+    sign = -1 if bits & 0x8000 else 1
+    e = (bits >> 7) & 0xFF
+    m = bits & 0x7F
+    assert e != 0xFF, "non-finite input"
+    if e == 0:
+        return sign * Fraction(m, 1 << 133)          # m * 2^-133
+    return sign * Fraction(128 + m, 128) * Fraction(2) ** (e - 127)
+
+
+def _f32_bits(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32)).view(np.uint32)
+
+
+# ---------------------------------------------------------------- unpacking
+
+def pin_unpack_hand_words(orc):
+    words, codes = [], []
+    for line in _golden_lines("unpack_words.txt"):
+        tok = line.split()
+        words.append(int(tok[0], 16))
+        codes.append([int(t) for t in tok[1:9]])
+    wq = np.array(words, dtype=np.uint32).reshape(len(words), 1)
+    got = orc.unpack(wq, 8)
+    assert np.array_equal(got, np.array(codes, dtype=np.uint8)), (got, codes)
+
+
+def pin_onehot_reads_codes(orc):
+    """x[m] = e_{k_m}, scale 1, bias 0  =>  y[m, n] = q[n, k_m] exactly."""
+    rng = np.random.default_rng(11)
+    M, N, K = 6, 40, 384
+    q = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    ks = rng.choice(K, size=M, replace=False)
+    x = np.zeros((M, K), np.float32)
+    x[np.arange(M), ks] = 1.0
+    G = K // 128
+    y = orc.matmul(synth.bf16_bits(x), synth.pack_nibbles(q),
+                   synth.bf16_bits(np.ones((N, G))), synth.bf16_bits(np.zeros((N, G))))
+    expect = synth.bf16_bits(q[:, ks].T.astype(np.float32))
+    assert np.array_equal(y, expect)
+
+
+# ---------------------------------------------------------------- closed forms
+
+def pin_identity_reproduces_x(orc):
+    """N = K, q = identity, scale 1, bias 0  =>  y == x bit for bit."""
+    rng = np.random.default_rng(12)
+    K = 256
+    M = 5
+    x = synth.make_x(rng, M, K, outliers=True)
+    q = np.eye(K, dtype=np.uint8)
+    G = K // 128
+    y = orc.matmul(x, synth.pack_nibbles(q), synth.bf16_bits(np.ones((K, G))),
+                   synth.bf16_bits(np.zeros((K, G))))
+    assert np.array_equal(y, x)
+
+
+def pin_bias_only(orc):
+    """All codes 0  =>  y[m,n] = sum_g b[n,g] * sum_{k in g} x[m,k] (integers: exact)."""
+    rng = np.random.default_rng(13)
+    M, N, K = 4, 9, 512
+    G = K // 128
+    xi = rng.integers(-3, 4, size=(M, K))
+    bi = rng.integers(-5, 6, size=(N, G))
+    si = rng.integers(1, 4, size=(N, G))
+    xsum = xi.reshape(M, G, 128).sum(-1)                # [M, G]
+    expect = xsum @ bi.T                                # [M, N]
+    y = orc.matmul(synth.bf16_bits(xi.astype(np.float32)),
+                   synth.pack_nibbles(np.zeros((N, K), np.uint8)),
+                   synth.bf16_bits(si.astype(np.float32)), synth.bf16_bits(bi.astype(np.float32)))
+    assert np.array_equal(y, synth.bf16_bits(expect.astype(np.float32)))
+
+
+def pin_all_ones_column_sums(orc):
+    """x = 1  =>  y[m,n] = sum_g (s[n,g] * sum_{k in g} q[n,k] + 128 * b[n,g])."""
+    from tolerance import compare
+    rng = np.random.default_rng(14)
+    M, N, K = 3, 33, 1024
+    G = K // 128
+    q = rng.integers(0, 16, size=(N, K)).astype(np.uint8)
+    s_bits = synth.bf16_bits(rng.uniform(0.001, 0.02, size=(N, G)))
+    b_bits = synth.bf16_bits(rng.uniform(-0.06, 0.0, size=(N, G)))
+    s = synth.bf16_to_f32(s_bits).astype(np.float64)
+    b = synth.bf16_to_f32(b_bits).astype(np.float64)
+    col = (s * q.reshape(N, G, 128).sum(-1) + 128.0 * b).sum(-1)      # [N] in float64
+    expect = synth.bf16_bits(np.broadcast_to(col, (M, N)).astype(np.float32))
+    y = orc.matmul(synth.bf16_bits(np.ones((M, K))), synth.pack_nibbles(q), s_bits, b_bits)
+    r = compare(y, expect)
+    assert r["fail"] == 0, r
+
+
+# ---------------------------------------------------------------- exact integers
+
+INTEGER_SHAPES = ((5, 24, 384), (1, 8, 128), (9, 17, 1024), (3, 1, 256), (2, 130, 640))
+
+
+def pin_integer_exact(orc):
+    """Integer inputs with exact FP32 sums: the accumulator equals int64
+    arithmetic and the output is that integer rounded once to BF16."""
+    for (M, N, K) in INTEGER_SHAPES:
+        p = synth.make_integer_problem(M, N, K)
+        G = K // 128
+        w = (p["si"][:, :, None] * p["qi"].reshape(N, G, 128) + p["bi"][:, :, None]).reshape(N, K)
+        expect = p["xi"] @ w.T
+        assert np.abs(expect).max() < 2 ** 24          # every FP32 partial sum is exact
+        y = orc.matmul(p["x"], p["wq"], p["scales"], p["biases"])
+        assert np.array_equal(y, synth.bf16_bits(expect.astype(np.float32))), (M, N, K)
+        acc = orc.matmul_f32(p["x"], p["wq"], p["scales"], p["biases"])
+        assert np.array_equal(acc, expect.astype(np.float32)), (M, N, K)
+
+
+# ---------------------------------------------------------------- rounding and accumulation
+
+def pin_bf16_rounding(orc):
+    f, e = [], []
+    for line in _golden_lines("bf16_rounding.txt"):
+        tok = line.split()
+        f.append(int(tok[0], 16))
+        e.append(int(tok[1], 16))
+    a = np.array(f, dtype=np.uint32).view(np.float32)
+    assert np.array_equal(orc.round_bf16(a), np.array(e, dtype=np.uint16))
+
+
+def pin_matmul_golden_cases(orc):
+    for line in _golden_lines("matmul_cases.txt"):
+        name, xs, qs, sb, bb, acc_bits, y_bits = [t.strip() for t in line.split("|")]
+        K = 128
+        x = np.zeros((1, K), np.uint16)
+        xv = _expand(xs)
+        x[0, :len(xv)] = xv
+        q = np.zeros((1, K), np.uint8)
+        qv = _expand(qs)
+        q[0, :len(qv)] = qv
+        s = np.array([[int(sb, 0)]], np.uint16)
+        b = np.array([[int(bb, 0)]], np.uint16)
+        wq = synth.pack_nibbles(q)
+        acc = orc.matmul_f32(x, wq, s, b)
+        y = orc.matmul(x, wq, s, b)
+        assert int(_f32_bits(acc)[0, 0]) == int(acc_bits, 0), (name, hex(int(_f32_bits(acc)[0, 0])))
+        assert int(y[0, 0]) == int(y_bits, 0), (name, hex(int(y[0, 0])))
+
+
+def pin_rational_brute_force(orc):
+    """Tiny random problems against exact rational arithmetic.
+
+    The FP32 accumulator must lie within the recursive-summation bound
+    (K + 2) * 2^-24 * sum_k |x_k w_k| of the exact value (the dequantised
+    weight itself carries one rounding, the product one, each sum one), and
+    the BF16 output within one BF16 ulp of the exact value.
+    """
+    from tolerance import ulp_bf16
+    u = Fraction(1, 1 << 24)
+    for (M, N, K, seed) in ((2, 3, 128, 1), (3, 2, 256, 2), (1, 4, 256, 3)):
+        rng = np.random.default_rng(seed)
+        x = synth.make_x(rng, M, K, outliers=True)
+        wq, s_bits, b_bits = synth.make_weights(rng, N, K)
+        G = K // 128
+        acc = orc.matmul_f32(x, wq, s_bits, b_bits)
+        y = orc.matmul(x, wq, s_bits, b_bits)
+        xf = [[_bits_to_fraction(int(v)) for v in row] for row in x]
+        sf = [[_bits_to_fraction(int(v)) for v in row] for row in s_bits]
+        bf = [[_bits_to_fraction(int(v)) for v in row] for row in b_bits]
+        for n in range(N):
+            w = []
+            for k in range(K):
+                code = (int(wq[n, k // 8]) >> (4 * (k % 8))) & 15
+                w.append(sf[n][k // 128] * code + bf[n][k // 128])
+            for m in range(M):
+                terms = [xf[m][k] * w[k] for k in range(K)]
+                exact = sum(terms, Fraction(0))
+                bound = (K + 2) * u * sum(abs(t) for t in terms)
+                err = abs(Fraction(float(acc[m, n])) - exact)
+                assert err <= bound, (m, n, float(err), float(bound))
+                ex = float(exact)
+                yv = float(synth.bf16_to_f32(y[m:m + 1, n])[0])
+                assert abs(yv - ex) <= float(ulp_bf16(np.array([ex]))[0]), (m, n, yv, ex)
+
+
+def pin_rejects_bad_k(orc):
+    x = np.zeros((1, 136), np.uint16)
+    wq = np.zeros((1, 17), np.uint32)
+    s = np.zeros((1, 1), np.uint16)
+    try:
+        orc.matmul(x, wq, s, s)
+    except ValueError:
+        return
+    raise AssertionError("K % 128 != 0 was accepted")
+
+
+ALL_PINS = (
+    pin_unpack_hand_words,
+    pin_onehot_reads_codes,
+    pin_identity_reproduces_x,
+    pin_bias_only,
+    pin_all_ones_column_sums,
+    pin_integer_exact,
+    pin_bf16_rounding,
+    pin_matmul_golden_cases,
+    pin_rational_brute_force,
+    pin_rejects_bad_k,
+)
+
+
+def run_all(orc) -> list[str]:
+    """Run every pin; return the names of those that failed."""
+    failed = []
+    for pin in ALL_PINS:
+        try:
+            pin(orc)
+        except AssertionError:
+            failed.append(pin.__name__)
+    return failed
+
+
+if __name__ == "__main__":
+    # used by the mutation test: run the pins against the library given on argv
+    import sys
+    from oracle import Oracle
+    bad = run_all(Oracle(sys.argv[1]))
+    print("FAILED:" + ",".join(bad))
+    sys.exit(1 if bad else 0)

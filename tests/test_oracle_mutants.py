@@ -1,0 +1,78 @@
+"""The pins must reject plausible mistakes in the oracle.
+
+Each case copies ``oracle/w4a16_oracle.c``, plants one mistake on the CPU (a
+reversed nibble order, a dropped bias, a transposed index, FP64 accumulation,
+fused multiply-adds, truncating output rounding, ...), builds the copy with the
+same flags and runs every pin against it in a child process.  At least one pin
+has to fail for each mutant; the real source must pass them all.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+import oracle
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+MUTANTS = {
+    "nibble_order_reversed": ("(word >> (4 * (k % 8)))", "(word >> (4 * (7 - k % 8)))"),
+    "code_mask_3_bits": ("& 15u);", "& 7u);"),
+    "word_index_stride": ("wq[n * (K / 8) + k / 8]", "wq[n * (K / 16) + k / 8]"),
+    "bias_dropped": ("const float w = sq + bi;", "const float w = sq;"),
+    "bias_sign": ("const float w = sq + bi;", "const float w = sq - bi;"),
+    "scale_dropped": ("const float sq = sc * q;", "const float sq = q;"),
+    "scale_group_index": ("bf16_to_f32(s[n * G + k / 128])", "bf16_to_f32(s[n * G + (k / 128) % 1])"),
+    "bias_from_scales": ("bf16_to_f32(b[n * G + k / 128])", "bf16_to_f32(s[n * G + k / 128])"),
+    "x_row_from_n": ("x[m * K + k]", "x[(n % 1 + m) * K + (k ^ 1)]"),
+    "fp64_accumulator": ("float acc = 0.0f;", "double acc = 0.0;"),
+    "truncating_round": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0u;"),
+    "ties_away": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0x8000u;"),
+    "k_descending": ("for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = K - 1; k >= 0; --k) {"),
+}
+
+
+def _build(tmp_path, name, src_text, extra_flags=()):
+    src = tmp_path / f"{name}.c"
+    src.write_text(src_text)
+    out = tmp_path / f"lib{name}.so"
+    flags = [f for f in oracle.CFLAGS if f != "-Werror"]   # a mutant may leave a variable unused
+    subprocess.run(["gcc", *flags, *extra_flags, str(src), "-o", str(out)], check=True)
+    return str(out)
+
+
+def _run_pins(lib):
+    env = dict(os.environ)
+    env["PYTHONPATH"] = os.pathsep.join([os.path.dirname(HERE), HERE, env.get("PYTHONPATH", "")])
+    env["OMP_NUM_THREADS"] = "1"
+    r = subprocess.run([sys.executable, os.path.join(HERE, "oracle_pins.py"), lib],
+                       capture_output=True, text=True, timeout=600, env=env)
+    return r.returncode, r.stdout + r.stderr
+
+
+def test_real_source_passes(tmp_path):
+    lib = _build(tmp_path, "real", open(oracle.SOURCE).read())
+    rc, out = _run_pins(lib)
+    assert rc == 0, out
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(tmp_path, name):
+    old, new = MUTANTS[name]
+    text = open(oracle.SOURCE).read()
+    assert old in text, f"mutation site for {name} not found"
+    lib = _build(tmp_path, name, text.replace(old, new))
+    rc, out = _run_pins(lib)
+    assert rc != 0, f"{name} survived every pin: {out}"
+
+
+def test_fused_multiply_add_is_caught(tmp_path):
+    """Building with contraction into FMAs must trip the unfused-product pin."""
+    try:
+        lib = _build(tmp_path, "fused", open(oracle.SOURCE).read(),
+                     extra_flags=("-ffp-contract=fast", "-mfma"))
+    except subprocess.CalledProcessError:
+        pytest.skip("compiler cannot target FMA here")
+    rc, out = _run_pins(lib)
+    assert rc != 0 and "pin_matmul_golden_cases" in out, out
