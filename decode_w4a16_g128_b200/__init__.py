@@ -1,0 +1,199 @@
+"""Python binding of libw4a16.so, the B200 W4A16 group-128 linear layer.
+
+Marshalling only: every function below checks tensor metadata, passes raw
+device pointers and the current CUDA stream to the C ABI declared in
+``include/w4a16.h`` and turns a non-zero status into ``W4A16Error``.  All
+arithmetic runs in the library's CUDA kernels; there is no fallback, and
+importing this package fails loudly when the shared library has not been
+built (``python -m decode_w4a16_g128_b200.build``).
+
+Tensors: ``x`` bf16 [M, K]; ``wq`` int32/uint32 [N, K/8] (eight 4-bit codes
+per word, low nibble first); ``scales``/``biases`` bf16 [N, K/128]; the result
+``y`` is bf16 [M, N].  All on the same CUDA device, contiguous.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIBRARY_PATH = os.path.join(_HERE, "libw4a16.so")
+
+OK = 0
+ERR_INVALID_ARG = 1
+ERR_UNSUPPORTED = 2
+ERR_MISALIGNED = 3
+ERR_CUDA = 4
+ERR_NO_MEMORY = 5
+ERR_DEVICE = 6
+ERR_TIMEOUT = 7
+
+PATH_AUTO = 0
+PATH_MATVEC = 1
+PATH_GEMM = 2
+
+FLAG_NO_PDL = 1
+
+
+class W4A16Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+class Options(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("splits", ctypes.c_int32), ("workers", ctypes.c_int32),
+                ("sm_count", ctypes.c_int32), ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+
+
+class PlanInfo(ctypes.Structure):
+    _fields_ = [("path", ctypes.c_int32), ("splits", ctypes.c_int32), ("grid_x", ctypes.c_int32),
+                ("grid_y", ctypes.c_int32), ("grid_z", ctypes.c_int32), ("block", ctypes.c_int32),
+                ("smem_bytes", ctypes.c_int32), ("cluster", ctypes.c_int32), ("tiles", ctypes.c_int64),
+                ("units", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIBRARY_PATH):
+        raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
+                          "`python -m decode_w4a16_g128_b200.build` (needs nvcc)")
+    lib = ctypes.CDLL(LIBRARY_PATH)
+    p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.w4a16_matmul.argtypes = [p, p, p, p, p, i64, i64, i64, p]
+    lib.w4a16_matmul_ex.argtypes = [p, p, p, p, p, i64, i64, i64, p, ctypes.POINTER(Options)]
+    lib.w4a16_matmul_last_rows.argtypes = [p, p, p, p, p, i64, i64, i64, i64, p]
+    lib.w4a16_plan.argtypes = [i64, i64, i64, ctypes.POINTER(Options), ctypes.POINTER(PlanInfo)]
+    lib.w4a16_device_status.argtypes = [p]
+    lib.w4a16_release.argtypes = []
+    lib.w4a16_release.restype = None
+    lib.w4a16_status_string.argtypes = [i32]
+    lib.w4a16_status_string.restype = ctypes.c_char_p
+    lib.w4a16_last_cuda_error.argtypes = []
+    lib.w4a16_version.argtypes = []
+    lib.w4a16_streamk_owner.argtypes = [i64, i64, i64]
+    lib.w4a16_streamk_owner.restype = i64
+    for name in ("w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan",
+                 "w4a16_device_status", "w4a16_last_cuda_error", "w4a16_version"):
+        getattr(lib, name).restype = i32
+    return lib
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.w4a16_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != OK:
+        raise W4A16Error(status, where)
+
+
+def _stream_handle(stream):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _check_tensors(x, wq, scales, biases, y):
+    import torch
+    if x.dtype != torch.bfloat16 or scales.dtype != torch.bfloat16 or biases.dtype != torch.bfloat16:
+        raise TypeError("x, scales and biases must be bfloat16")
+    if wq.dtype not in (torch.int32, torch.uint32):
+        raise TypeError("wq must be int32 or uint32 (packed codes)")
+    for name, t in (("x", x), ("wq", wq), ("scales", scales), ("biases", biases)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    M, K = x.shape
+    N = wq.shape[0]
+    if tuple(wq.shape) != (N, K // 8) or tuple(scales.shape) != (N, K // 128) or \
+            tuple(biases.shape) != (N, K // 128):
+        raise ValueError(f"shape mismatch: x {tuple(x.shape)}, wq {tuple(wq.shape)}, "
+                         f"scales {tuple(scales.shape)}, biases {tuple(biases.shape)}")
+    if y is not None and (y.dtype != torch.bfloat16 or not y.is_cuda or not y.is_contiguous()):
+        raise ValueError("y must be a contiguous bfloat16 CUDA tensor")
+    return M, N, K
+
+
+def w4a16_matmul(x, wq, scales, biases, y=None, stream=None):
+    """y = x . dequant(wq)^T on the current (or given) CUDA stream; returns y."""
+    import torch
+    M, N, K = _check_tensors(x, wq, scales, biases, y)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif tuple(y.shape) != (M, N):
+        raise ValueError("y must be [M, N]")
+    _check(lib.w4a16_matmul(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
+                            _stream_handle(stream)), "w4a16_matmul")
+    return y
+
+
+def make_options(path=PATH_AUTO, splits=0, workers=0, sm_count=0, flags=0) -> Options:
+    return Options(int(path), int(splits), int(workers), int(sm_count), int(flags))
+
+
+def w4a16_matmul_ex(x, wq, scales, biases, y=None, stream=None, path=PATH_AUTO, splits=0, workers=0,
+                    flags=0):
+    """w4a16_matmul with a forced path / split count / worker count."""
+    import torch
+    M, N, K = _check_tensors(x, wq, scales, biases, y)
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif tuple(y.shape) != (M, N):
+        raise ValueError("y must be [M, N]")
+    opt = make_options(path, splits, workers, 0, flags)
+    _check(lib.w4a16_matmul_ex(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
+                               _stream_handle(stream), ctypes.byref(opt)), "w4a16_matmul_ex")
+    return y
+
+
+def w4a16_matmul_last_rows(x, wq, scales, biases, keep: int, y=None, stream=None):
+    """Project only the last ``keep`` rows of x (0 = every row); returns y [keep, N]."""
+    import torch
+    M, N, K = _check_tensors(x, wq, scales, biases, None)
+    rows = M if keep == 0 else keep
+    if y is None:
+        y = torch.empty((rows, N), dtype=torch.bfloat16, device=x.device)
+    elif tuple(y.shape) != (rows, N):
+        raise ValueError("y must be [keep, N]")
+    _check(lib.w4a16_matmul_last_rows(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(y), M,
+                                      int(keep), N, K, _stream_handle(stream)),
+           "w4a16_matmul_last_rows")
+    return y
+
+
+def w4a16_plan(M: int, N: int, K: int, path=PATH_AUTO, splits=0, workers=0, sm_count=0) -> dict:
+    opt = make_options(path, splits, workers, sm_count)
+    info = PlanInfo()
+    _check(lib.w4a16_plan(M, N, K, ctypes.byref(opt), ctypes.byref(info)), "w4a16_plan")
+    return {name: getattr(info, name) for name, _ in PlanInfo._fields_}
+
+
+def w4a16_device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    return lib.w4a16_device_status(_stream_handle(stream))
+
+
+def w4a16_release() -> None:
+    lib.w4a16_release()
+
+
+def w4a16_version() -> int:
+    return lib.w4a16_version()
+
+
+def w4a16_streamk_owner(units: int, workers: int, u: int) -> int:
+    return lib.w4a16_streamk_owner(units, workers, u)
+
+
+__all__ = [
+    "w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan", "w4a16_device_status",
+    "w4a16_release", "w4a16_version", "w4a16_streamk_owner", "status_string", "W4A16Error", "Options",
+    "PlanInfo", "make_options", "lib", "LIBRARY_PATH",
+]

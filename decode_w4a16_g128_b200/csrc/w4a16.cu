@@ -1,0 +1,422 @@
+// w4a16.cu - the C ABI declared in include/w4a16.h, built as ONE translation
+// unit with every kernel of the library (so the device status word has a
+// single definition).  Host code here validates arguments, plans the launch,
+// owns the split bookkeeping workspace and encodes the TMA tensor maps.
+// There is no host fallback: every output element is computed by a kernel.
+#include "w4a16.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <utility>
+
+#include "matvec.cuh"
+
+namespace w4a16 {
+namespace {
+
+constexpr int kVersion = 100;          // 0.1.0
+constexpr int kMatvecWarps = 8;        // consumer warps of the matvec CTA (16 rows each)
+using MvCfg = mv::Cfg<kMatvecWarps>;
+constexpr int kMinTickets = 1 << 16;   // ticket slots allocated up front (grows on demand)
+
+std::atomic<int> g_last_cuda_error{0};
+
+int cuda_fail(cudaError_t e) {
+    g_last_cuda_error.store(static_cast<int>(e));
+    return W4A16_ERR_CUDA;
+}
+
+struct DeviceInfo {
+    bool ready = false;
+    int status = W4A16_OK;
+    int sms = 0;
+    PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
+};
+
+struct Workspace {
+    float *partials = nullptr;
+    size_t partial_floats = 0;
+    int *tickets = nullptr;
+    int64_t ticket_count = 0;
+};
+
+std::mutex g_mu;
+std::map<int, DeviceInfo> g_devices;
+std::map<std::pair<int, void *>, Workspace> g_workspaces;
+
+// Per-device one-time set-up: capability check, SM count, driver entry point,
+// kernel attributes.  Caller holds g_mu.
+int device_setup(int dev, DeviceInfo **out) {
+    DeviceInfo &d = g_devices[dev];
+    if (!d.ready) {
+        int major = 0, minor = 0;
+        cudaError_t e = cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+        if (e == cudaSuccess) e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (major != 10 || minor != 0) {
+            d.status = W4A16_ERR_DEVICE;
+        } else {
+            void *fn = nullptr;
+            cudaDriverEntryPointQueryResult q{};
+            e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
+            if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
+            d.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            e = cudaFuncSetAttribute(mv::matvec_kernel<kMatvecWarps>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, MvCfg::kSmemBytes);
+            if (e != cudaSuccess) return cuda_fail(e);
+        }
+        d.ready = true;
+    }
+    *out = &d;
+    return d.status;
+}
+
+int current_device(int *dev) {
+    cudaError_t e = cudaGetDevice(dev);
+    return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+}
+
+// Workspace of (device, stream), grown to at least the requested sizes.  A
+// stream that is being captured cannot allocate, so growth there is refused.
+int workspace_get(int dev, void *stream, size_t partial_floats, int64_t tickets, Workspace **out) {
+    Workspace &w = g_workspaces[{dev, stream}];
+    const bool grow_p = w.partial_floats < partial_floats;
+    const bool grow_t = w.ticket_count < tickets;
+    if (grow_p || grow_t) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        cudaError_t e = cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (cap != cudaStreamCaptureStatusNone) return W4A16_ERR_UNSUPPORTED;
+        e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));   // old buffers may be in use
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (grow_p) {
+            cudaFree(w.partials);
+            w.partials = nullptr;
+            w.partial_floats = 0;
+            if (cudaMalloc(&w.partials, partial_floats * sizeof(float)) != cudaSuccess) {
+                cudaGetLastError();
+                return W4A16_ERR_NO_MEMORY;
+            }
+            w.partial_floats = partial_floats;
+        }
+        if (grow_t) {
+            const int64_t count = std::max<int64_t>(tickets, kMinTickets);
+            cudaFree(w.tickets);
+            w.tickets = nullptr;
+            w.ticket_count = 0;
+            if (cudaMalloc(&w.tickets, count * sizeof(int)) != cudaSuccess) {
+                cudaGetLastError();
+                return W4A16_ERR_NO_MEMORY;
+            }
+            e = cudaMemset(w.tickets, 0, count * sizeof(int));
+            if (e != cudaSuccess) return cuda_fail(e);
+            w.ticket_count = count;
+        }
+    }
+    *out = &w;
+    return W4A16_OK;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool overlaps(const void *a, size_t na, const void *b, size_t nb) {
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a), b0 = reinterpret_cast<uintptr_t>(b);
+    return a0 < b0 + nb && b0 < a0 + na;
+}
+
+struct Problem {
+    const void *x;
+    const uint32_t *wq;
+    const void *scales;
+    const void *biases;
+    void *y;
+    int64_t M, N, K;
+};
+
+int validate(const Problem &p) {
+    if (p.M < 0 || p.N < 0 || p.K < 0) return W4A16_ERR_INVALID_ARG;
+    if (p.K % 128 != 0) return W4A16_ERR_UNSUPPORTED;
+    if (p.M >= (int64_t(1) << 31) || p.N >= (int64_t(1) << 31) || p.K >= (int64_t(1) << 31))
+        return W4A16_ERR_UNSUPPORTED;
+    if (p.M == 0 || p.N == 0) return W4A16_OK;
+    if (!p.y) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(p.y)) return W4A16_ERR_MISALIGNED;
+    if (p.K == 0) return W4A16_OK;
+    if (!p.x || !p.wq || !p.scales || !p.biases) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(p.x) || !aligned16(p.wq) || !aligned16(p.scales) || !aligned16(p.biases))
+        return W4A16_ERR_MISALIGNED;
+    const size_t ny = size_t(p.M) * p.N * 2;
+    if (overlaps(p.y, ny, p.x, size_t(p.M) * p.K * 2) || overlaps(p.y, ny, p.wq, size_t(p.N) * p.K / 2) ||
+        overlaps(p.y, ny, p.scales, size_t(p.N) * (p.K / 128) * 2) ||
+        overlaps(p.y, ny, p.biases, size_t(p.N) * (p.K / 128) * 2))
+        return W4A16_ERR_INVALID_ARG;
+    return W4A16_OK;
+}
+
+int choose_path(int64_t M, const w4a16_options *opt, int *path) {
+    const int req = opt ? opt->path : W4A16_PATH_AUTO;
+    if (req == W4A16_PATH_AUTO) {
+        *path = M <= mv::kMaxM ? W4A16_PATH_MATVEC : W4A16_PATH_GEMM;
+    } else if (req == W4A16_PATH_MATVEC) {
+        if (M > mv::kMaxM) return W4A16_ERR_UNSUPPORTED;
+        *path = W4A16_PATH_MATVEC;
+    } else if (req == W4A16_PATH_GEMM) {
+        *path = W4A16_PATH_GEMM;
+    } else {
+        return W4A16_ERR_INVALID_ARG;
+    }
+    return W4A16_OK;
+}
+
+int validate_options(const w4a16_options *opt) {
+    if (!opt) return W4A16_OK;
+    if (opt->splits < 0 || opt->splits > 16 || opt->workers < 0 || opt->sm_count < 0) return W4A16_ERR_INVALID_ARG;
+    if (opt->flags & ~1) return W4A16_ERR_INVALID_ARG;
+    return W4A16_OK;
+}
+
+// ------------------------------------------------------------------ planning
+
+void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, w4a16_plan_info *pl) {
+    (void)M;
+    const int64_t G = K / 128;
+    const int64_t tiles = (N + MvCfg::kRows - 1) / MvCfg::kRows;
+    const int64_t units = tiles * G;
+    int64_t workers = (opt && opt->workers > 0) ? opt->workers : sms;
+    workers = std::max<int64_t>(1, std::min<int64_t>(workers, units));
+    std::memset(pl, 0, sizeof(*pl));
+    pl->path = W4A16_PATH_MATVEC;
+    pl->splits = 1;
+    pl->grid_x = static_cast<int32_t>(workers);
+    pl->grid_y = pl->grid_z = 1;
+    pl->block = MvCfg::kThreads;
+    pl->smem_bytes = MvCfg::kSmemBytes;
+    pl->cluster = 1;
+    pl->tiles = tiles;
+    pl->units = units;
+    pl->workspace_bytes = int64_t(workers) * 2 * MvCfg::kRows * 8 * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
+}
+
+int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a16_plan_info *pl) {
+    int path = 0;
+    int rc = choose_path(M, opt, &path);
+    if (rc) return rc;
+    if (path == W4A16_PATH_MATVEC) {
+        plan_matvec(M, N, K, sms, opt, pl);
+        return W4A16_OK;
+    }
+    return W4A16_ERR_UNSUPPORTED;   // tensor-core GEMM path not built yet
+}
+
+// ------------------------------------------------------------------ launches
+
+int encode_2d(DeviceInfo *d, CUtensorMap *map, CUtensorMapDataType type, const void *base, uint64_t inner,
+              uint64_t outer, uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer,
+              CUtensorMapSwizzle swizzle) {
+    const cuuint64_t dims[2] = {inner, outer};
+    const cuuint64_t strides[1] = {row_bytes};
+    const cuuint32_t box[2] = {box_inner, box_outer};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = d->encode(map, type, 2, const_cast<void *>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        g_last_cuda_error.store(static_cast<int>(r));
+        return W4A16_ERR_CUDA;
+    }
+    return W4A16_OK;
+}
+
+int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan_info &pl, void *stream,
+                  bool pdl) {
+    CUtensorMap tm_w, tm_x;
+    int rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16, MvCfg::kRows,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+    rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, mv::kXCols,
+                   static_cast<uint32_t>(p.M), CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+    mv::Params kp;
+    kp.scales = static_cast<const uint16_t *>(p.scales);
+    kp.biases = static_cast<const uint16_t *>(p.biases);
+    kp.y = static_cast<uint16_t *>(p.y);
+    kp.partials = ws->partials;
+    kp.tickets = ws->tickets;
+    kp.M = static_cast<int>(p.M);
+    kp.N = static_cast<int>(p.N);
+    kp.G = static_cast<int>(p.K / 128);
+    kp.tiles = static_cast<int>(pl.tiles);
+    kp.units = pl.units;
+    kp.workers = pl.grid_x;
+    kp.pdl = pdl ? 1 : 0;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid_x, 1, 1);
+    cfg.blockDim = dim3(pl.block, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mv::matvec_kernel<kMatvecWarps>, tm_w, tm_x, kp);
+    return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+}
+
+int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
+    int rc = validate(p);
+    if (rc) return rc;
+    rc = validate_options(opt);
+    if (rc) return rc;
+    int path = 0;
+    rc = choose_path(p.M, opt, &path);
+    if (rc) return rc;
+    if (p.M == 0 || p.N == 0) return W4A16_OK;
+
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo *d = nullptr;
+    rc = device_setup(dev, &d);
+    if (rc) return rc;
+    if (p.K == 0) {   // an empty sum: every output is +0
+        cudaError_t e = cudaMemsetAsync(p.y, 0, size_t(p.M) * p.N * 2, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+    }
+    w4a16_plan_info pl;
+    rc = plan(p.M, p.N, p.K, opt, d->sms, &pl);
+    if (rc) return rc;
+    const bool pdl = !(opt && (opt->flags & 1));
+    if (pl.path == W4A16_PATH_MATVEC) {
+        Workspace *ws = nullptr;
+        rc = workspace_get(dev, stream, size_t(pl.grid_x) * 2 * MvCfg::kRows * 8, pl.tiles, &ws);
+        if (rc) return rc;
+        return launch_matvec(d, ws, p, pl, stream, pdl);
+    }
+    return W4A16_ERR_UNSUPPORTED;
+}
+
+}  // namespace
+}  // namespace w4a16
+
+using namespace w4a16;
+
+extern "C" {
+
+int w4a16_matmul(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *y, int64_t M,
+                 int64_t N, int64_t K, void *stream) {
+    return matmul_impl(Problem{x, wq, scales, biases, y, M, N, K}, stream, nullptr);
+}
+
+int w4a16_matmul_ex(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *y, int64_t M,
+                    int64_t N, int64_t K, void *stream, const w4a16_options *opt) {
+    return matmul_impl(Problem{x, wq, scales, biases, y, M, N, K}, stream, opt);
+}
+
+int w4a16_matmul_last_rows(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *y,
+                           int64_t M, int64_t keep, int64_t N, int64_t K, void *stream) {
+    if (M < 0 || keep < 0 || keep > M || K < 0) return W4A16_ERR_INVALID_ARG;
+    if (keep == 0) keep = M;
+    const char *xs = static_cast<const char *>(x);
+    if (xs) xs += (M - keep) * K * 2;   // the last `keep` rows of x
+    return matmul_impl(Problem{xs, wq, scales, biases, y, keep, N, K}, stream, nullptr);
+}
+
+int w4a16_plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, w4a16_plan_info *out) {
+    if (!out) return W4A16_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return W4A16_ERR_INVALID_ARG;
+    if (K % 128 != 0) return W4A16_ERR_UNSUPPORTED;
+    int rc = validate_options(opt);
+    if (rc) return rc;
+    int sms = opt ? opt->sm_count : 0;
+    if (sms <= 0) {
+        int dev = 0;
+        rc = current_device(&dev);
+        if (rc) return rc;
+        std::lock_guard<std::mutex> lock(g_mu);
+        DeviceInfo *d = nullptr;
+        rc = device_setup(dev, &d);
+        if (rc) return rc;
+        sms = d->sms;
+    }
+    if (M == 0 || N == 0 || K == 0) {
+        std::memset(out, 0, sizeof(*out));
+        int path = 0;
+        rc = choose_path(M, opt, &path);
+        out->path = path;
+        return rc;
+    }
+    return plan(M, N, K, opt, sms, out);
+}
+
+int w4a16_device_status(void *stream) {
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    int status = 0;
+    e = cudaMemcpyFromSymbol(&status, g_status, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (status == 0) return W4A16_OK;
+    // A kernel gave up: clear the word and the split bookkeeping of this device.
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_status, &zero, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e);
+    int dev = 0;
+    if (current_device(&dev)) return W4A16_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mu);
+    for (auto &kv : g_workspaces) {
+        if (kv.first.first != dev || !kv.second.tickets) continue;
+        e = cudaMemset(kv.second.tickets, 0, kv.second.ticket_count * sizeof(int));
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    return W4A16_ERR_TIMEOUT;
+}
+
+void w4a16_release(void) {
+    std::lock_guard<std::mutex> lock(g_mu);
+    int cur = 0;
+    cudaGetDevice(&cur);
+    for (auto &kv : g_workspaces) {
+        cudaSetDevice(kv.first.first);
+        cudaDeviceSynchronize();
+        cudaFree(kv.second.partials);
+        cudaFree(kv.second.tickets);
+    }
+    g_workspaces.clear();
+    cudaSetDevice(cur);
+}
+
+const char *w4a16_status_string(int status) {
+    switch (status) {
+        case W4A16_OK: return "ok";
+        case W4A16_ERR_INVALID_ARG: return "invalid argument";
+        case W4A16_ERR_UNSUPPORTED: return "unsupported size or option";
+        case W4A16_ERR_MISALIGNED: return "pointer not 16-byte aligned";
+        case W4A16_ERR_CUDA: return "CUDA call failed";
+        case W4A16_ERR_NO_MEMORY: return "workspace allocation failed";
+        case W4A16_ERR_DEVICE: return "device is not compute capability 10.0";
+        case W4A16_ERR_TIMEOUT: return "a kernel abandoned a bounded wait";
+        default: return "unknown status";
+    }
+}
+
+int w4a16_last_cuda_error(void) { return g_last_cuda_error.load(); }
+
+int w4a16_version(void) { return kVersion; }
+
+int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u) {
+    if (units <= 0 || workers <= 0 || workers > units || u < 0 || u >= units) return -1;
+    return mv::streamk_owner(units, workers, u);
+}
+
+}  // extern "C"

@@ -1,0 +1,163 @@
+/*
+ * w4a16.h - C ABI of the B200 (sm_100a) W4A16 group-128 linear layer.
+ *
+ *     y[M,N] = x[M,K] . dequant(wq)^T,   dequant: w[n,k] = s[n,k/128] * q[n,k] + b[n,k/128]
+ *
+ * The operation is the quantised linear layer of tiny-llm "Week 2 Day 6:
+ * SIMD-Matrix Prefill": 4-bit weights with group size 128, BF16 activations,
+ * BF16 quantisation parameters and BF16 output, FP32 matrix accumulators
+ * (introduction), one scale and one bias per 128 reduction values (Task 3), a
+ * matvec schedule for M <= 8 and a tiled matrix schedule for M > 8 behind one
+ * unchanged interface (Task 1), a split-K successor for under-filled grids
+ * (Task 5), and last-row logits (Task 4).
+ *
+ * Data layout (all row-major, contiguous, DEVICE memory owned by the caller):
+ *   x       bf16   [M, K]
+ *   wq      uint32 [N, K/8]   code q[n,k] = (wq[n*(K/8) + k/8] >> (4*(k%8))) & 15
+ *                             (eight 4-bit codes per word, k % 8 == 0 in bits 0-3)
+ *   scales  bf16   [N, K/128]
+ *   biases  bf16   [N, K/128]
+ *   y       bf16   [M, N]     written; must not overlap any input
+ * Every pointer must be 16-byte aligned.  K must be a multiple of 128.
+ *
+ * Numerics: products and sums in FP32, each 128-wide group's scale and bias
+ * applied in FP32, one BF16 round-to-nearest-even per output.  The result
+ * matches the plain FP32 definition to within one BF16 ulp (+1e-3 absolute);
+ * the summation order differs from it.  Identical inputs and sizes give
+ * bit-identical outputs on the same device model (no atomics decide the order
+ * of any floating-point sum).
+ *
+ * Execution: work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ * default stream) on the CURRENT device; calls return without synchronising.
+ * No call allocates in steady state; the first call on a (device, stream)
+ * pair allocates a small library-owned workspace (see w4a16_release), so
+ * that first call must not happen during stream capture.  Calls on different
+ * streams use different workspaces and may overlap.
+ *
+ * Errors: every entry point validates its arguments on the host and returns a
+ * status code without launching anything when they are invalid.  Kernels
+ * never trap: a kernel that gives up on a bounded wait records
+ * W4A16_ERR_TIMEOUT in a device-side status word, which w4a16_device_status
+ * reports.
+ */
+#ifndef W4A16_H
+#define W4A16_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+enum w4a16_status_code {
+    W4A16_OK = 0,
+    W4A16_ERR_INVALID_ARG = 1,  /* null pointer with non-empty sizes, negative size, bad option  */
+    W4A16_ERR_UNSUPPORTED = 2,  /* K % 128 != 0, or a size beyond the supported range            */
+    W4A16_ERR_MISALIGNED = 3,   /* a pointer that is not 16-byte aligned                          */
+    W4A16_ERR_CUDA = 4,         /* a CUDA runtime call failed (see w4a16_last_cuda_error)         */
+    W4A16_ERR_NO_MEMORY = 5,    /* the library-owned workspace could not be allocated             */
+    W4A16_ERR_DEVICE = 6,       /* the current device is not compute capability 10.0             */
+    W4A16_ERR_TIMEOUT = 7       /* a kernel abandoned a bounded wait (from w4a16_device_status)   */
+};
+
+/* Kernel paths (w4a16_options.path, w4a16_plan_info.path). */
+enum w4a16_path {
+    W4A16_PATH_AUTO = 0,        /* M <= 8: matvec; M > 8: tensor-core GEMM (Task 1 dispatch rule) */
+    W4A16_PATH_MATVEC = 1,      /* weight-streaming matvec, M <= 8 only                           */
+    W4A16_PATH_GEMM = 2         /* tcgen05 tensor-core GEMM, any M >= 1                            */
+};
+
+/*
+ * y = x . dequant(wq)^T.  Arguments as in the layout block above.
+ * M == 0 or N == 0: returns W4A16_OK and launches nothing.
+ * Sizes: 0 <= M, N < 2^31, 0 <= K < 2^31 with K % 128 == 0.
+ * Ownership: all buffers belong to the caller and must stay valid until the
+ * enqueued work completes.
+ */
+int w4a16_matmul(const void *x, const uint32_t *wq, const void *scales,
+                 const void *biases, void *y, int64_t M, int64_t N, int64_t K,
+                 void *stream);
+
+/*
+ * Last-rows projection ("logits_to_keep", tiny-llm "Week 2 Day 6: SIMD-Matrix
+ * Prefill", Task 4): y[keep, N] = x[M-keep : M, :] . dequant(wq)^T.
+ * keep == 0 keeps every row (y is [M, N]); 0 < keep <= M keeps the last keep
+ * rows.  No kernel of its own: the rows are selected by offsetting x, then
+ * w4a16_matmul runs with M' = keep.  keep > M or keep < 0: W4A16_ERR_INVALID_ARG.
+ */
+int w4a16_matmul_last_rows(const void *x, const uint32_t *wq, const void *scales,
+                           const void *biases, void *y, int64_t M, int64_t keep,
+                           int64_t N, int64_t K, void *stream);
+
+/* Options for the explicit entry points; zero-initialised means "automatic". */
+typedef struct w4a16_options {
+    int32_t path;      /* enum w4a16_path                                                  */
+    int32_t splits;    /* GEMM: K splits (1..16), each a contiguous run of 128-groups; 0 = auto */
+    int32_t workers;   /* matvec: persistent CTAs sharing the (row-tile x group) units; 0 = auto */
+    int32_t sm_count;  /* w4a16_plan only: SM count to plan for; 0 = query the current device   */
+    int32_t flags;     /* bit 0: disable programmatic dependent launch                       */
+    int32_t reserved[3];
+} w4a16_options;
+
+/*
+ * w4a16_matmul with explicit options (tests and benchmarks force a path or a
+ * split count through it).  opt == NULL behaves like w4a16_matmul.  Forcing
+ * the matvec path with M > 8 returns W4A16_ERR_UNSUPPORTED.
+ */
+int w4a16_matmul_ex(const void *x, const uint32_t *wq, const void *scales,
+                    const void *biases, void *y, int64_t M, int64_t N, int64_t K,
+                    void *stream, const w4a16_options *opt);
+
+/* What a call of the given size would launch (host-side planning only). */
+typedef struct w4a16_plan_info {
+    int32_t path;            /* enum w4a16_path chosen                                  */
+    int32_t splits;          /* GEMM K splits (cluster size along K); 1 for the matvec  */
+    int32_t grid_x, grid_y, grid_z;
+    int32_t block;           /* threads per CTA                                         */
+    int32_t smem_bytes;      /* dynamic shared memory per CTA                           */
+    int32_t cluster;         /* CTAs per cluster (1 = no cluster)                       */
+    int64_t tiles;           /* output tiles                                            */
+    int64_t units;           /* matvec: (row tile x 128-group) work units               */
+    int64_t workspace_bytes; /* library workspace the call needs                        */
+} w4a16_plan_info;
+
+/*
+ * Fill *out with the launch plan for an M x N x K call.  Performs no CUDA call
+ * when opt->sm_count > 0, so it also runs on machines without a GPU.
+ */
+int w4a16_plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt,
+               w4a16_plan_info *out);
+
+/*
+ * Synchronise `stream`, then read and clear the device-side status word of the
+ * current device.  Returns W4A16_OK, W4A16_ERR_TIMEOUT (a kernel abandoned a
+ * bounded wait; its outputs are undefined and the library's split bookkeeping
+ * has been reset) or W4A16_ERR_CUDA.
+ */
+int w4a16_device_status(void *stream);
+
+/* Free every library-owned workspace on every device (synchronises them). */
+void w4a16_release(void);
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *w4a16_status_string(int status);
+
+/* cudaError_t value of the most recent failed CUDA call made by the library. */
+int w4a16_last_cuda_error(void);
+
+/* ABI version: major * 10000 + minor * 100 + patch. */
+int w4a16_version(void);
+
+/*
+ * Stream-K bookkeeping of the matvec, exported for host-side tests: the CTA
+ * (0 <= c < workers) whose contiguous unit range contains unit u when `units`
+ * units are split over `workers` CTAs (CTA c owns [c*units/workers,
+ * (c+1)*units/workers)).  Returns -1 for arguments out of range.
+ */
+int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* W4A16_H */

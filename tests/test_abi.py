@@ -1,0 +1,127 @@
+"""Host-side checks of the C ABI that need no GPU: every symbol the header
+declares is exported, argument validation returns its status before touching
+memory or CUDA, and the launch planning / stream-K bookkeeping are consistent."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import decode_w4a16_g128_b200 as w4
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "w4a16.h")
+lib = w4.lib
+P = ctypes.c_void_p
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(w4a16_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_header_symbols_exported():
+    names = declared_functions()
+    assert len(names) >= 10
+    for name in names:
+        assert hasattr(lib, name), f"{name} declared in include/w4a16.h but not exported"
+
+
+def test_version_and_strings():
+    assert w4.w4a16_version() >= 100
+    for code in range(8):
+        assert w4.status_string(code)
+    assert w4.status_string(99) == "unknown status"
+
+
+def mm(x, wq, s, b, y, M, N, K):
+    return lib.w4a16_matmul(P(x), P(wq), P(s), P(b), P(y), M, N, K, P(0))
+
+
+A = 0x10000  # a 16-byte aligned address that is never dereferenced: validation fails first
+
+
+@pytest.mark.parametrize("M,N,K,status", [
+    (-1, 8, 128, w4.ERR_INVALID_ARG),
+    (1, -8, 128, w4.ERR_INVALID_ARG),
+    (1, 8, -128, w4.ERR_INVALID_ARG),
+    (1, 8, 100, w4.ERR_UNSUPPORTED),
+    (1, 8, 136, w4.ERR_UNSUPPORTED),
+    (1, 2 ** 31, 128, w4.ERR_UNSUPPORTED),
+])
+def test_bad_sizes(M, N, K, status):
+    assert mm(A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x400000, M, N, K) == status
+
+
+def test_empty_outputs_need_no_gpu():
+    assert mm(0, 0, 0, 0, 0, 0, 8, 128) == w4.OK
+    assert mm(0, 0, 0, 0, 0, 4, 0, 128) == w4.OK
+
+
+def test_null_and_misaligned_pointers():
+    good = [A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x400000]
+    for i in range(5):
+        args = list(good)
+        args[i] = 0
+        assert mm(*args, 2, 8, 256) == w4.ERR_INVALID_ARG
+        args = list(good)
+        args[i] += 8
+        assert mm(*args, 2, 8, 256) == w4.ERR_MISALIGNED
+
+
+def test_output_overlapping_input_is_rejected():
+    # y placed inside x
+    assert mm(A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x100, 4, 8, 256) == w4.ERR_INVALID_ARG
+
+
+def test_last_rows_argument_checks():
+    f = lib.w4a16_matmul_last_rows
+    args = (P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000), P(A + 0x400000))
+    assert f(*args, 4, 5, 8, 256, P(0)) == w4.ERR_INVALID_ARG     # keep > M
+    assert f(*args, 4, -1, 8, 256, P(0)) == w4.ERR_INVALID_ARG    # keep < 0
+    assert f(*args, 0, 0, 8, 256, P(0)) == w4.OK                  # nothing to do
+
+
+def test_bad_options():
+    opt = w4.make_options(path=7)
+    assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
+                               P(A + 0x400000), 2, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_INVALID_ARG
+    opt = w4.make_options(path=w4.PATH_MATVEC)
+    assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
+                               P(A + 0x400000), 9, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_UNSUPPORTED
+    opt = w4.make_options(splits=17)
+    assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
+                               P(A + 0x400000), 2, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_INVALID_ARG
+
+
+def test_dispatch_rule():
+    """M <= 8 streams weights through the matvec; larger M goes to the tensor-core GEMM."""
+    for M in range(1, 9):
+        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148)["path"] == w4.PATH_MATVEC
+
+
+@pytest.mark.parametrize("N,K", [(1024, 2560), (4096, 2560), (2560, 4096), (9728, 2560), (2560, 9728),
+                                 (151936, 2560), (1000, 256), (8, 128)])
+def test_matvec_plan(N, K):
+    pl = w4.w4a16_plan(1, N, K, sm_count=148)
+    rows = 16 * (pl["block"] // 32 - 1)
+    assert pl["tiles"] == -(-N // rows)
+    assert pl["units"] == pl["tiles"] * (K // 128)
+    assert 1 <= pl["grid_x"] <= min(148, pl["units"])
+    assert pl["smem_bytes"] <= 227 * 1024
+
+
+def test_streamk_owner_matches_brute_force():
+    for U in list(range(1, 40)) + [640, 1520, 23740]:
+        for Pw in sorted({1, 2, 3, 7, 37, 148, U}):
+            if Pw > U:
+                continue
+            owner = []
+            for c in range(Pw):
+                owner += [c] * ((c + 1) * U // Pw - c * U // Pw)
+            assert len(owner) == U
+            for u in range(0, U, max(1, U // 97)):
+                assert w4.w4a16_streamk_owner(U, Pw, u) == owner[u], (U, Pw, u)
+    assert w4.w4a16_streamk_owner(10, 11, 0) == -1
+    assert w4.w4a16_streamk_owner(10, 2, 10) == -1
