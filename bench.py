@@ -1,0 +1,474 @@
+#!/usr/bin/env python3
+"""Throughput of the W4A16 group-128 linear layer on B200.
+
+Default workload (one "step"): the decode matvec over the seven Qwen3-4B
+projections (q 2560->4096, k/v 2560->1024, o 4096->2560, gate/up 2560->9728,
+down 9728->2560) for each batch size M in {1, 2, 4, 8}: 28 calls of
+w4a16_matmul on synthetic seeded inputs (x ~ N(0,1) BF16, W ~ N(0,0.02)
+quantised to 4 bits per 128-group).
+
+Metric: algorithmic bytes per second (GB/s) and FLOP/s, against the HBM
+roofline.  Algorithmic bytes per call = N*K/2 (codes) + 4*N*K/128 (BF16 scale
+and bias) + 2*M*K (x) + 2*M*N (y); FLOPs = 2*M*N*K.
+
+Timing: the 28 calls of a step are captured once in a CUDA graph per weight
+set; two weight sets of 215 MB each (every (M, projection) pair has its own
+copy) alternate between steps, so the working set between two uses of the
+same bytes is 430 MB, far above the 126 MB L2.  W >= 3 warm-up steps, then K
+timed steps between CUDA events on the launching stream, with a barrier and a
+device synchronise on both sides; the step time is the max over ranks.
+
+Also reported: the oracle timed on the host cores (cpu_baseline), an
+end-to-end figure through the Python/C ABI with host buffers (H2D of the
+step's activations, 28 calls, D2H of the outputs), SM clocks sampled during
+the timed region, and the roofline of the matvec kernel.
+
+`--impl reference` times the CPU oracle on the same workload (a bounded
+sample of each step's output columns) and prints the same line with
+"impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import w4a16_synth as synth  # noqa: E402
+
+METRIC = "W4A16 matmul TFLOP/s & GB/s on 1 B200 vs roofline fraction (M=1..2048)"
+DECODE_M = (1, 2, 4, 8)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ("decode_w4a16_g128_b200/csrc/matvec.cuh", "decode_w4a16_g128_b200/csrc/ptx.cuh")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "matvec_decode_traffic.json")
+
+
+def algo_bytes(M, N, K):
+    return N * K // 2 + 4 * N * K // 128 + 2 * M * K + 2 * M * N
+
+
+def decode_calls():
+    return [(M, name, K, N) for M in DECODE_M for (name, K, N) in synth.QWEN3_4B_PROJECTIONS]
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return dict(FALLBACK_PEAKS, source="fallback")
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for rel in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic():
+    """Per-launch DRAM bytes from the committed ncu capture, if it matches this kernel."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+    except (OSError, ValueError):
+        return None
+    if d.get("kernel_sha") != kernel_hash():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ---------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi samples every 200 ms while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=5)
+        sm, mx, reasons = [], None, set()
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        for line in self.lines:
+            f = [t.strip() for t in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for name, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return None
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- distributed
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_group(world, backend):
+    import torch.distributed as dist
+    from datetime import timedelta
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend, timeout=timedelta(seconds=300))
+    return dist
+
+
+def max_over_ranks(value, world, device):
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ---------------------------------------------------------------- workload
+
+def make_host_inputs():
+    """Seeded inputs of the decode step: one weight set per projection, one x per (M, projection)."""
+    weights = {}
+    for (name, K, N) in synth.QWEN3_4B_PROJECTIONS:
+        rng = synth.shape_rng(0, N, K, seed=0)
+        weights[name] = synth.make_weights(rng, N, K)
+    xs = {}
+    for (M, name, K, N) in decode_calls():
+        xs[(M, name)] = synth.make_x(synth.shape_rng(M, N, K, seed=1), M, K)
+    return weights, xs
+
+
+def cpu_sample(weights, xs, frac):
+    """The oracle over the first ceil(frac*N) output columns of every call of a step."""
+    import oracle
+    nbytes = 0
+    t0 = time.perf_counter()
+    for (M, name, K, N) in decode_calls():
+        wq, s, b = weights[name]
+        n = max(1, int(math.ceil(N * frac)))
+        oracle.matmul(xs[(M, name)], wq[:n], s[:n], b[:n])
+        nbytes += algo_bytes(M, n, K)
+    return nbytes, time.perf_counter() - t0
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    import oracle
+    weights, xs = make_host_inputs()
+    frac = args.ref_fraction
+    for _ in range(args.warmup):
+        cpu_sample(weights, xs, frac)
+    total_b, total_t = 0, 0.0
+    for _ in range(args.steps):
+        b, t = cpu_sample(weights, xs, frac)
+        total_b += b
+        total_t += t
+    gbs = total_b / total_t / 1e9
+    ms = total_t / args.steps * 1e3
+    sample = (f"oracle on the first {frac:g} of the output columns of each of the 28 calls "
+              f"(M in {{1,2,4,8}} x 7 projections) per step")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+        "data": "synthetic", "config": workload_config(),
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def workload_config():
+    return {
+        "workload": "decode matvec: M in {1,2,4,8} x Qwen3-4B projections q 2560->4096, k/v 2560->1024, "
+                    "o 4096->2560, gate/up 2560->9728, down 9728->2560 (28 calls per step)",
+        "group_size": 128, "bits": 4,
+        "l2": "inputs larger than L2: two rotating weight sets of 215 MB (430 MB between reuses)",
+        "timing": "CUDA graph of the 28 calls per step, CUDA events on the launching stream",
+        "flags": "W4A16_FLAG_STATIC_WEIGHTS (weights streamed while the previous call finishes)",
+    }
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import decode_w4a16_g128_b200 as w4
+
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        init_group(world, "nccl")
+    pk = peaks()
+
+    weights, xs = make_host_inputs()
+    calls = decode_calls()
+    nsets = 2
+
+    def dev_bf16(a):
+        return torch.from_numpy(a.view(np.int16)).to(device).view(torch.bfloat16)
+
+    base_w = {name: (torch.from_numpy(wq.view(np.int32)).to(device), dev_bf16(s), dev_bf16(b))
+              for name, (wq, s, b) in weights.items()}
+    sets = []
+    for _ in range(nsets):
+        entries = []
+        for (M, name, K, N) in calls:
+            wq, s, b = base_w[name]
+            x = dev_bf16(xs[(M, name)])
+            y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+            entries.append((x, wq.clone(), s.clone(), b.clone(), y))
+        sets.append(entries)
+    del base_w
+    step_bytes = sum(algo_bytes(M, N, K) for (M, _, K, N) in calls)
+    step_flops = sum(2 * M * N * K for (M, _, K, N) in calls)
+
+    stream = torch.cuda.Stream(device)
+
+    # weights are static across the step: let each call start streaming them while the
+    # previous call finishes (programmatic dependent launch); x is read after it completes
+    flags = w4.FLAG_STATIC_WEIGHTS
+
+    def launch_set(entries):
+        for (x, wq, s, b, y) in entries:
+            w4.w4a16_matmul_ex(x, wq, s, b, y=y, flags=flags)
+
+    # warm the workspace of the capture stream, then capture one graph per set
+    with torch.cuda.stream(stream):
+        for entries in sets:
+            launch_set(entries)
+    stream.synchronize()
+    graphs = []
+    for entries in sets:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            launch_set(entries)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    if w4.w4a16_device_status(stream) != w4.OK:
+        raise RuntimeError("device status not ok after capture")
+
+    if args.mode == "profile":
+        # exactly two eager steps (56 launches) for ncu: skip 28, capture the next 28
+        with torch.cuda.stream(stream):
+            launch_set(sets[0])
+            launch_set(sets[0])
+        torch.cuda.synchronize()
+        return 0
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            graphs[i % nsets].replay()
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        start.record(stream)
+        for i in range(args.steps):
+            graphs[i % nsets].replay()
+        end.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clocks = sampler.stop()
+    ms_total = start.elapsed_time(end)
+    ms_total = max_over_ranks(ms_total, world, device)
+    ms_step = ms_total / args.steps
+    status = w4.w4a16_device_status(stream)
+    if status != w4.OK:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    gbs = step_bytes * world / (ms_step * 1e-3) / 1e9
+    tflops = step_flops * world / (ms_step * 1e-3) / 1e12
+    launches = len(calls)
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9      # per GPU: bytes per launch / mean launch time
+    traffic = recorded_traffic()
+
+    # end to end through the binding: H2D of this step's activations, 28 eager calls, D2H of outputs
+    host_x = [torch.from_numpy(xs[(M, name)].view(np.int16)).pin_memory() for (M, name, K, N) in calls]
+    host_y = [torch.empty((M, N), dtype=torch.int16).pin_memory() for (M, name, K, N) in calls]
+    h2d = sum(t.numel() * 2 for t in host_x)
+    d2h = sum(t.numel() * 2 for t in host_y)
+
+    def e2e_step(entries):
+        for hx, hy, (x, wq, s, b, y) in zip(host_x, host_y, entries):
+            x.view(torch.int16).copy_(hx, non_blocking=True)
+            w4.w4a16_matmul_ex(x, wq, s, b, y=y, flags=flags)
+            hy.copy_(y.view(torch.int16), non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup):
+            e2e_step(sets[i % nsets])
+    torch.cuda.synchronize()
+    barrier(world)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for i in range(args.steps):
+            e2e_step(sets[i % nsets])
+        e1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
+    e2e_gbs = step_bytes * world / (e2e_ms * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        import oracle
+        nb, t = cpu_sample(weights, xs, 1.0)
+        cpu = {"value": round(nb / t / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+               "sample": "one full decode step (all 28 calls) through the C oracle, OpenMP over outputs"}
+
+    if args.detail and rank == 0:
+        detail(args, sets[0], calls, stream, pk)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 5), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": workload_config(),
+            "tflops": round(tflops, 3),
+            "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(achieved / pk["hbm_gbs"], 4), "traffic": traffic,
+                         "peak_source": pk["source"], "kernel": "w4a16::mv::matvec_kernel<8>",
+                         "algorithmic_bytes_per_launch": round(step_bytes / launches)},
+            "cpu_baseline": cpu,
+            "e2e": {"value": round(e2e_gbs, 2), "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": launches * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.destroy_process_group()
+    return 0
+
+
+def detail(args, entries, calls, stream, pk):
+    """Per-call times (graph of 20 back-to-back repeats of one call over 8 weight copies)."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    rows = []
+    for (x, wq, s, b, y), (M, name, K, N) in zip(entries, calls):
+        copies = [(wq.clone(), s.clone(), b.clone()) for _ in range(max(2, int(400e6 // (N * K // 2)) + 1))]
+        copies = copies[:32]
+        reps = 64
+        with torch.cuda.stream(stream):
+            for (cw, cs, cb) in copies:
+                w4.w4a16_matmul_ex(x, cw, cs, cb, y=y, flags=w4.FLAG_STATIC_WEIGHTS)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(reps):
+                cw, cs, cb = copies[i % len(copies)]
+                w4.w4a16_matmul_ex(x, cw, cs, cb, y=y, flags=w4.FLAG_STATIC_WEIGHTS)
+        with torch.cuda.stream(stream):
+            g.replay()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(5):
+                g.replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        us = e0.elapsed_time(e1) * 1e3 / (5 * reps)
+        gb = algo_bytes(M, N, K) / (us * 1e-6) / 1e9
+        rows.append({"M": M, "proj": name, "N": N, "K": K, "us": round(us, 3), "GB/s": round(gb, 1),
+                     "frac_hbm": round(gb / pk["hbm_gbs"], 3)})
+        del g, copies
+    out = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ROOT
+    with open(os.path.join(out, "bench_detail.json"), "w") as f:
+        json.dump(rows, f, indent=1)
+    for r in rows:
+        print(json.dumps(r), file=sys.stderr)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
+    ap.add_argument("--mode", choices=("bench", "profile"), default="bench")
+    ap.add_argument("--detail", action="store_true", help="also time every call on its own")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--ref-fraction", type=float, default=0.125,
+                    help="reference arm: fraction of each call's output columns per step")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.mode == "bench":
+        ap.error("--warmup must be at least 3")
+    world, rank, local = dist_setup(args)
+    if args.impl == "reference":
+        return run_reference(args, world, rank)
+    return run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

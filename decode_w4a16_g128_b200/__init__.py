@@ -33,6 +33,7 @@ PATH_MATVEC = 1
 PATH_GEMM = 2
 
 FLAG_NO_PDL = 1
+FLAG_STATIC_WEIGHTS = 2
 
 
 class W4A16Error(RuntimeError):

@@ -23,9 +23,13 @@ namespace w4a16 {
 namespace {
 
 constexpr int kVersion = 100;          // 0.1.0
-constexpr int kMatvecWarps = 8;        // consumer warps of the matvec CTA (16 rows each)
-using MvCfg = mv::Cfg<kMatvecWarps>;
 constexpr int kMinTickets = 1 << 16;   // ticket slots allocated up front (grows on demand)
+// Shared memory a matvec CTA may use so that a CTA of the next launch in the
+// stream fits beside it on the same SM (programmatic dependent launch).
+constexpr long long kMatvecPairBudget = 112 * 1024;
+constexpr long long kMatvecSoloBudget = 220 * 1024;
+constexpr int kMatvecMaxStages = 10;
+constexpr int kMatvecMinStages = 3;
 
 std::atomic<int> g_last_cuda_error{0};
 
@@ -70,8 +74,10 @@ int device_setup(int dev, DeviceInfo **out) {
             e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
             if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
             d.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-            e = cudaFuncSetAttribute(mv::matvec_kernel<kMatvecWarps>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, MvCfg::kSmemBytes);
+            e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     int(kMatvecSoloBudget));
+            if (e == cudaSuccess)   // one carveout for every launch: no reconfiguration between them
+                e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e != cudaSuccess) return cuda_fail(e);
         }
         d.ready = true;
@@ -180,16 +186,38 @@ int choose_path(int64_t M, const w4a16_options *opt, int *path) {
 int validate_options(const w4a16_options *opt) {
     if (!opt) return W4A16_OK;
     if (opt->splits < 0 || opt->splits > 16 || opt->workers < 0 || opt->sm_count < 0) return W4A16_ERR_INVALID_ARG;
-    if (opt->flags & ~1) return W4A16_ERR_INVALID_ARG;
+    if (opt->flags & ~(W4A16_FLAG_NO_PDL | W4A16_FLAG_STATIC_WEIGHTS)) return W4A16_ERR_INVALID_ARG;
     return W4A16_OK;
 }
 
 // ------------------------------------------------------------------ planning
 
+// Ring depth and scale/bias slab slots of the matvec for G groups: two slab
+// slots and as many stages as fit the pair budget; one slot when two do not
+// leave kMatvecMinStages; a solo-CTA budget, then no slab, for very long K.
+void matvec_smem_plan(int64_t G, int *stages, int *slots, long long *bytes) {
+    auto fit = [&](long long budget, int nslots) {
+        for (int st = kMatvecMaxStages; st >= kMatvecMinStages; --st)
+            if (mv::smem_bytes(st, nslots, G) <= budget) return st;
+        return 0;
+    };
+    int st = 0, sl = 0;
+    if ((st = fit(kMatvecPairBudget, 2))) sl = 2;
+    else if ((st = fit(kMatvecPairBudget, 1))) sl = 1;
+    else if ((st = fit(kMatvecSoloBudget, 1))) sl = 1;
+    else { st = fit(kMatvecPairBudget, 0); sl = 0; }
+    *stages = st;
+    *slots = sl;
+    *bytes = mv::smem_bytes(st, sl, G);
+}
+
 void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, w4a16_plan_info *pl) {
     (void)M;
     const int64_t G = K / 128;
-    const int64_t tiles = (N + MvCfg::kRows - 1) / MvCfg::kRows;
+    int stages = 0, slots = 0;
+    long long smem = 0;
+    matvec_smem_plan(G, &stages, &slots, &smem);
+    const int64_t tiles = (N + mv::kRows - 1) / mv::kRows;
     const int64_t units = tiles * G;
     int64_t workers = (opt && opt->workers > 0) ? opt->workers : sms;
     workers = std::max<int64_t>(1, std::min<int64_t>(workers, units));
@@ -198,12 +226,12 @@ void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
     pl->splits = 1;
     pl->grid_x = static_cast<int32_t>(workers);
     pl->grid_y = pl->grid_z = 1;
-    pl->block = MvCfg::kThreads;
-    pl->smem_bytes = MvCfg::kSmemBytes;
+    pl->block = mv::kThreads;
+    pl->smem_bytes = static_cast<int32_t>(smem);
     pl->cluster = 1;
     pl->tiles = tiles;
     pl->units = units;
-    pl->workspace_bytes = int64_t(workers) * 2 * MvCfg::kRows * 8 * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
+    pl->workspace_bytes = int64_t(workers) * 2 * mv::kRows * 8 * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
 }
 
 int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a16_plan_info *pl) {
@@ -237,12 +265,14 @@ int encode_2d(DeviceInfo *d, CUtensorMap *map, CUtensorMapDataType type, const v
 }
 
 int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan_info &pl, void *stream,
-                  bool pdl) {
+                  bool pdl, bool static_weights) {
     CUtensorMap tm_w, tm_x;
-    int rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16, MvCfg::kRows,
-                       CU_TENSOR_MAP_SWIZZLE_NONE);
+    // codes: [N, K/8] uint32, box of 2 groups (32 words = 128 B) x 128 rows, 128-byte swizzle
+    int rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2,
+                       16 * mv::kGroupsPerStage, mv::kRows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
-    rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, mv::kXCols,
+    // x viewed as [M, K/2] pairs of BF16: box of 264 BF16 (132 pairs) x M rows
+    rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.x, p.K / 2, p.M, p.K * 2, mv::kXCols / 2,
                    static_cast<uint32_t>(p.M), CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
     mv::Params kp;
@@ -257,7 +287,10 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     kp.tiles = static_cast<int>(pl.tiles);
     kp.units = pl.units;
     kp.workers = pl.grid_x;
-    kp.pdl = pdl ? 1 : 0;
+    long long smem = 0;
+    matvec_smem_plan(kp.G, &kp.stages, &kp.slab_slots, &smem);
+    kp.slab_array_bytes = static_cast<int>(mv::slab_array_bytes(kp.G));
+    kp.flags = static_weights ? mv::kFlagStaticWeights : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid_x, 1, 1);
@@ -269,7 +302,7 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, mv::matvec_kernel<kMatvecWarps>, tm_w, tm_x, kp);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mv::matvec_kernel, tm_w, tm_x, kp);
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
@@ -297,12 +330,13 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     w4a16_plan_info pl;
     rc = plan(p.M, p.N, p.K, opt, d->sms, &pl);
     if (rc) return rc;
-    const bool pdl = !(opt && (opt->flags & 1));
+    const bool pdl = !(opt && (opt->flags & W4A16_FLAG_NO_PDL));
+    const bool static_weights = opt && (opt->flags & W4A16_FLAG_STATIC_WEIGHTS);
     if (pl.path == W4A16_PATH_MATVEC) {
         Workspace *ws = nullptr;
-        rc = workspace_get(dev, stream, size_t(pl.grid_x) * 2 * MvCfg::kRows * 8, pl.tiles, &ws);
+        rc = workspace_get(dev, stream, size_t(pl.grid_x) * 2 * mv::kRows * 8, pl.tiles, &ws);
         if (rc) return rc;
-        return launch_matvec(d, ws, p, pl, stream, pdl);
+        return launch_matvec(d, ws, p, pl, stream, pdl, pdl && static_weights);
     }
     return W4A16_ERR_UNSUPPORTED;
 }

@@ -95,9 +95,23 @@ typedef struct w4a16_options {
     int32_t splits;    /* GEMM: K splits (1..16), each a contiguous run of 128-groups; 0 = auto */
     int32_t workers;   /* matvec: persistent CTAs sharing the (row-tile x group) units; 0 = auto */
     int32_t sm_count;  /* w4a16_plan only: SM count to plan for; 0 = query the current device   */
-    int32_t flags;     /* bit 0: disable programmatic dependent launch                       */
+    int32_t flags;     /* W4A16_FLAG_* bits                                                 */
     int32_t reserved[3];
 } w4a16_options;
+
+/*
+ * w4a16_options.flags.
+ * W4A16_FLAG_NO_PDL: launch without programmatic dependent launch (the kernel
+ *   then starts only after the previous work in the stream has finished).
+ * W4A16_FLAG_STATIC_WEIGHTS: the caller promises that wq, scales and biases are
+ *   not written by work still pending in the stream, so the kernel may start
+ *   streaming them before the preceding kernel completes (x is always read
+ *   after it).  This is the usual situation for model weights in a decode loop.
+ */
+enum w4a16_flags {
+    W4A16_FLAG_NO_PDL = 1,
+    W4A16_FLAG_STATIC_WEIGHTS = 2
+};
 
 /*
  * w4a16_matmul with explicit options (tests and benchmarks force a path or a

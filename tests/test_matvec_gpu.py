@@ -124,3 +124,31 @@ def test_last_rows_matvec():
     assert y.shape == (1, 4096)
     sub = dict(prob, x=np.ascontiguousarray(prob["x"][5:6]))
     assert_close(bits(y), oracle_y(sub))
+
+
+@pytest.mark.parametrize("flags", [0, 1, 2, 3])
+@pytest.mark.parametrize("M,N,K", [(4, 2560, 9728), (1, 1000, 2560), (8, 129, 384)])
+def test_launch_flags(flags, M, N, K):
+    prob = synth.make_integer_problem(M, N, min(K, 1024)) if K <= 1024 else synth.make_problem(M, N, K)
+    got = run(prob, flags=flags)
+    if K <= 1024:
+        assert np.array_equal(got, oracle_y(prob))
+    else:
+        assert_close(got, oracle_y(prob), f"flags={flags}")
+
+
+@pytest.mark.parametrize("workers", [1, 2, 3, 148])
+def test_single_slab_slot_recycling(workers):
+    """K = 9728 keeps one scale/bias slab slot, so CTAs spanning several row
+    tiles must recycle it; a single worker walks all 20 tiles in sequence."""
+    prob = synth.make_problem(2, 2560, 9728, outliers=True)
+    assert_close(run(prob, path=w4.PATH_MATVEC, workers=workers, flags=w4.FLAG_STATIC_WEIGHTS),
+                 oracle_y(prob), f"workers={workers}")
+
+
+def test_long_k_without_slab():
+    """K = 65536 (512 groups) is too long for a scale/bias slab: values come from global memory."""
+    prob = synth.make_problem(3, 200, 65536)
+    assert w4.w4a16_plan(3, 200, 65536)["smem_bytes"] <= 112 * 1024
+    assert_close(run(prob), oracle_y(prob), "K=65536")
+
