@@ -73,8 +73,9 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_version.argtypes = []
     lib.w4a16_streamk_owner.argtypes = [i64, i64, i64]
     lib.w4a16_streamk_owner.restype = i64
+    lib.w4a16_matvec_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, p]
     for name in ("w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan",
-                 "w4a16_device_status", "w4a16_last_cuda_error", "w4a16_version"):
+                 "w4a16_device_status", "w4a16_last_cuda_error", "w4a16_version", "w4a16_matvec_noalloc"):
         getattr(lib, name).restype = i32
     return lib
 
@@ -169,6 +170,21 @@ def w4a16_matmul_last_rows(x, wq, scales, biases, keep: int, y=None, stream=None
     return y
 
 
+NOALLOC_MAX_N = 1048576
+
+
+def w4a16_matvec_noalloc(x, wq, scales, biases, y, stream=None):
+    """The matvec (M <= 8) without any allocation, for callers that cannot allocate
+    device memory: its split-row scratch is a fixed array inside the library, so
+    calls that can overlap on the GPU must be serialised.  y must be given."""
+    M, N, K = _check_tensors(x, wq, scales, biases, y)
+    if tuple(y.shape) != (M, N):
+        raise ValueError("y must be [M, N]")
+    _check(lib.w4a16_matvec_noalloc(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
+                                    _stream_handle(stream)), "w4a16_matvec_noalloc")
+    return y
+
+
 def w4a16_plan(M: int, N: int, K: int, path=PATH_AUTO, splits=0, workers=0, sm_count=0) -> dict:
     opt = make_options(path, splits, workers, sm_count)
     info = PlanInfo()
@@ -195,6 +211,6 @@ def w4a16_streamk_owner(units: int, workers: int, u: int) -> int:
 
 __all__ = [
     "w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan", "w4a16_device_status",
-    "w4a16_release", "w4a16_version", "w4a16_streamk_owner", "status_string", "W4A16Error", "Options",
+    "w4a16_release", "w4a16_version", "w4a16_streamk_owner", "w4a16_matvec_noalloc", "status_string", "W4A16Error", "Options",
     "PlanInfo", "make_options", "lib", "LIBRARY_PATH",
 ]

@@ -341,6 +341,62 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     return W4A16_ERR_UNSUPPORTED;
 }
 
+// ------------------------------------------------------------------ allocation-free matvec
+
+// Scratch of w4a16_matvec_noalloc: FP32 partials of up to kNoAllocWorkers CTAs,
+// then one ticket per 128-row tile for up to W4A16_NOALLOC_MAX_N rows.
+constexpr int kNoAllocWorkers = 160;
+constexpr size_t kNoAllocPartialBytes = size_t(kNoAllocWorkers) * 2 * mv::kRows * 8 * sizeof(float);
+constexpr int64_t kNoAllocTiles = W4A16_NOALLOC_MAX_N / mv::kRows;
+static_assert(kNoAllocPartialBytes + kNoAllocTiles * sizeof(int) == W4A16_NOALLOC_SCRATCH_BYTES,
+              "header and scratch layout disagree");
+static __device__ __align__(256) unsigned char g_noalloc_scratch[W4A16_NOALLOC_SCRATCH_BYTES];
+
+std::map<int, unsigned char *> g_noalloc_ptr;   // device address of the array, per device
+
+int noalloc_matvec(const Problem &p, void *stream) {
+    if (p.M < 0 || p.N < 0 || p.K < 0) return W4A16_ERR_INVALID_ARG;
+    if (p.M > mv::kMaxM || p.N > W4A16_NOALLOC_MAX_N) return W4A16_ERR_UNSUPPORTED;   // beyond the scratch
+    int rc = validate(p);
+    if (rc) return rc;
+    if (p.M == 0 || p.N == 0) return W4A16_OK;
+    int dev = 0;
+    rc = current_device(&dev);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo *d = nullptr;
+    rc = device_setup(dev, &d);
+    if (rc) return rc;
+    if (p.K == 0) {
+        cudaError_t e = cudaMemsetAsync(p.y, 0, size_t(p.M) * p.N * 2, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+    }
+    auto it = g_noalloc_ptr.find(dev);
+    if (it == g_noalloc_ptr.end()) {
+        // In host code the array's name is only a stand-in: look up its address on
+        // this device (the current one) before handing it to a kernel.
+        void *ptr = nullptr;
+        cudaError_t e = cudaGetSymbolAddress(&ptr, g_noalloc_scratch);
+        if (e != cudaSuccess || !ptr) return cuda_fail(e);
+        it = g_noalloc_ptr.emplace(dev, static_cast<unsigned char *>(ptr)).first;
+    }
+    w4a16_plan_info pl;
+    w4a16_options opt = {};
+    opt.path = W4A16_PATH_MATVEC;
+    opt.workers = std::min(d->sms, kNoAllocWorkers);
+    plan_matvec(p.M, p.N, p.K, d->sms, &opt, &pl);
+    if (pl.tiles > kNoAllocTiles || pl.grid_x > kNoAllocWorkers) return W4A16_ERR_UNSUPPORTED;
+    Workspace ws;
+    ws.partials = reinterpret_cast<float *>(it->second);
+    ws.partial_floats = kNoAllocPartialBytes / sizeof(float);
+    ws.tickets = reinterpret_cast<int *>(it->second + kNoAllocPartialBytes);
+    ws.ticket_count = kNoAllocTiles;
+    // the tickets of this call must start at zero whatever an earlier call left behind
+    cudaError_t e = cudaMemsetAsync(ws.tickets, 0, size_t(pl.tiles) * sizeof(int), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return launch_matvec(d, &ws, p, pl, stream, /*pdl=*/true, /*static_weights=*/false);
+}
+
 }  // namespace
 }  // namespace w4a16
 
@@ -451,6 +507,11 @@ int w4a16_version(void) { return kVersion; }
 int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u) {
     if (units <= 0 || workers <= 0 || workers > units || u < 0 || u >= units) return -1;
     return mv::streamk_owner(units, workers, u);
+}
+
+int w4a16_matvec_noalloc(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *y,
+                         int64_t M, int64_t N, int64_t K, void *stream) {
+    return noalloc_matvec(Problem{x, wq, scales, biases, y, M, N, K}, stream);
 }
 
 }  // extern "C"

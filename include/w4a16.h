@@ -170,6 +170,33 @@ int w4a16_version(void);
  */
 int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u);
 
+/*
+ * Allocation-free matvec (M <= 8).  The pages have no counterpart: this entry
+ * point exists for callers that cannot allocate device memory -- code running
+ * under a memory pool or allocator that owns all device memory, inside a
+ * capture or real-time loop where cudaMalloc is forbidden, or in processes
+ * without the right to create allocations.  It runs the same kernel as
+ * w4a16_matmul on the matvec path, but the scratch it needs for rows split
+ * across CTAs (FP32 partial sums and per-tile tickets) lives in one
+ * file-scope device array of W4A16_NOALLOC_SCRATCH_BYTES that every GPU
+ * loading the library holds until the process exits.  The call itself
+ * allocates nothing (no cudaMalloc, no allocating library routine).
+ *
+ * Limits: 1 <= M <= 8 and N <= W4A16_NOALLOC_MAX_N; larger sizes return
+ * W4A16_ERR_UNSUPPORTED without launching.  Other arguments, layouts and
+ * errors are those of w4a16_matmul.
+ * Set-up: the first call on a device looks up the array's device address
+ * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * Sharing: every call uses the same array and clears its tickets on `stream`
+ * before launching, so calls whose kernels can overlap on the GPU (different
+ * streams without ordering) race and give undefined results; serialise them.
+ */
+#define W4A16_NOALLOC_MAX_N 1048576
+#define W4A16_NOALLOC_SCRATCH_BYTES 1343488
+int w4a16_matvec_noalloc(const void *x, const uint32_t *wq, const void *scales,
+                         const void *biases, void *y, int64_t M, int64_t N,
+                         int64_t K, void *stream);
+
 #ifdef __cplusplus
 }
 #endif
