@@ -134,9 +134,11 @@ __global__ void __maxnreg__(112)
     matvec_kernel(const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_x,
                   const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    // 1 KB alignment for the swizzled code tiles (x is loaded through a uint32 view of
-    // [M, K/2] pairs, so its 264-column box is a legal 132-element box)
-    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    // 1 KB alignment for the swizzled code tiles, by offsetting within the shared
+    // array (so the compiler still knows every access below is a shared-memory one).
+    // x is loaded through a uint32 view of [M, K/2] pairs, so its 264-column box is a
+    // legal 132-element box.
+    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     const int S = p.stages;
     const int XR = static_cast<int>(xs_ring(S));
     uint8_t *slab_base = smem + S * kStageBytes;
@@ -284,9 +286,13 @@ __global__ void __maxnreg__(112)
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     int tile_seq = -1, prev_t = -1;
     const uint16_t *sA = nullptr, *sB = nullptr, *bA = nullptr, *bB = nullptr;   // scale/bias rows
+    const int first_tile = static_cast<int>(u0 / G);
     StageWalker wk;
     wk.start(u0, u1, G);
-    for (int i = 0; wk.n; ++i, wk.next()) {
+    int s = 0, xslot = 0;                 // ring positions of stage i
+    uint32_t ph = 0, xph = 0;             // their phase parities
+    for (int i = 0; wk.n; ++i, wk.next(), (++s == S ? (s = 0, ph ^= 1u) : 0u),
+             (++xslot == XR ? (xslot = 0, xph ^= 1u) : 0u)) {
         const int t = wk.t;
         const long long first_row = static_cast<long long>(t) * kRows;
         if (t != prev_t) {
@@ -312,8 +318,7 @@ __global__ void __maxnreg__(112)
                 sA = p.scales + nA * G; sB = p.scales + nB * G; bA = p.biases + nA * G; bB = p.biases + nB * G;
             }
         }
-        const int s = i % S;
-        mbar_wait(&full[s], (i / S) & 1);
+        mbar_wait(&full[s], ph);
         const uint8_t *st = smem + s * kStageBytes;
         const int ng = wk.n;
         const int g0 = wk.g;
@@ -366,7 +371,6 @@ __global__ void __maxnreg__(112)
             }
 
         // X = sum of x over each group of this stage: computed by the stage's duty warp
-        const int xslot = i % XR;
         float *xs_slot = xs_base + xslot * (kGroupsPerStage * kMaxM);
         if ((i % kWarps) == warp) {
             float xa[2][4] = {}, xb[2][4] = {};
@@ -405,7 +409,7 @@ __global__ void __maxnreg__(112)
             }
 
         // epilogue: rows rA (d0, d1) and rB (d2, d3); x rows 2tq, 2tq+1
-        mbar_wait(&xs_full[xslot], (i / XR) & 1);
+        mbar_wait(&xs_full[xslot], xph);
 #pragma unroll
         for (int j = 0; j < 2; ++j) {
             if (j >= ng) break;
@@ -432,7 +436,7 @@ __global__ void __maxnreg__(112)
         bool write = true;
         if (!(tile_first >= u0 && tile_last < u1)) {
             // split tile: publish this CTA's partial, take a ticket, last arriver reduces
-            const int slot = (t == static_cast<int>(u0 / G)) ? 0 : 1;
+            const int slot = (t == first_tile) ? 0 : 1;
             float *mine = p.partials + (cta * 2 + slot) * (kRows * 8);
             *reinterpret_cast<float2 *>(mine + rA * 8 + 2 * tq) = make_float2(acc[0], acc[1]);
             *reinterpret_cast<float2 *>(mine + rB * 8 + 2 * tq) = make_float2(acc[2], acc[3]);
@@ -449,6 +453,10 @@ __global__ void __maxnreg__(112)
             named_bar_sync(1, kWarps * 32);
             write = *ticket_flag != 0;
             if (write) {
+                // Every contributor after the first starts inside this tile, so its partial
+                // is in slot 0; the first one uses slot 1 unless its range starts exactly at
+                // the tile's first unit.
+                const int first_slot = (c_first * U / P == tile_first) ? 0 : 1;
                 out[0] = out[1] = out[2] = out[3] = 0.f;
                 for (long long cb = c_first; cb <= c_last; cb += kFixupBatch) {
                     float2 v[kFixupBatch][2];
@@ -456,7 +464,7 @@ __global__ void __maxnreg__(112)
                     for (int j = 0; j < kFixupBatch; ++j) {   // issue every load of the batch first
                         const long long cc = cb + j;
                         if (cc <= c_last) {
-                            const int cslot = (t == static_cast<int>((cc * U / P) / G)) ? 0 : 1;
+                            const int cslot = (cc == c_first) ? first_slot : 0;
                             const float *part = p.partials + (cc * 2 + cslot) * (kRows * 8);
                             v[j][0] = __ldcg(reinterpret_cast<const float2 *>(part + rA * 8 + 2 * tq));
                             v[j][1] = __ldcg(reinterpret_cast<const float2 *>(part + rB * 8 + 2 * tq));
