@@ -17,6 +17,7 @@
 #include <mutex>
 #include <utility>
 
+#include "gemm.cuh"
 #include "matvec.cuh"
 
 namespace w4a16 {
@@ -78,6 +79,8 @@ int device_setup(int dev, DeviceInfo **out) {
                                      int(kMatvecSoloBudget));
             if (e == cudaSuccess)   // one carveout for every launch: no reconfiguration between them
                 e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gm::kSmemBytes);
             if (e != cudaSuccess) return cuda_fail(e);
         }
         d.ready = true;
@@ -234,6 +237,28 @@ void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
     pl->workspace_bytes = int64_t(workers) * 2 * mv::kRows * 8 * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
 }
 
+// Tensor-core GEMM: 128 x 128 output tiles; K split into `splits` contiguous runs
+// of 128-groups (forced by the options, else 1).
+void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, w4a16_plan_info *pl) {
+    (void)sms;
+    const int64_t G = K / 128;
+    const int64_t tm = (M + gm::BM - 1) / gm::BM, tn = (N + gm::BN - 1) / gm::BN;
+    int64_t splits = (opt && opt->splits > 0) ? opt->splits : 1;
+    splits = std::max<int64_t>(1, std::min<int64_t>(splits, G));
+    std::memset(pl, 0, sizeof(*pl));
+    pl->path = W4A16_PATH_GEMM;
+    pl->splits = static_cast<int32_t>(splits);
+    pl->grid_x = static_cast<int32_t>(tn);
+    pl->grid_y = static_cast<int32_t>(tm);
+    pl->grid_z = static_cast<int32_t>(splits);
+    pl->block = gm::kThreads;
+    pl->smem_bytes = gm::kSmemBytes;
+    pl->cluster = 1;
+    pl->tiles = tm * tn;
+    pl->units = tm * tn * G;
+    pl->workspace_bytes = 0;
+}
+
 int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a16_plan_info *pl) {
     int path = 0;
     int rc = choose_path(M, opt, &path);
@@ -242,7 +267,11 @@ int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a
         plan_matvec(M, N, K, sms, opt, pl);
         return W4A16_OK;
     }
-    return W4A16_ERR_UNSUPPORTED;   // tensor-core GEMM path not built yet
+    if (N >= (int64_t(1) << 31) / 1 || (N + gm::BN - 1) / gm::BN > 0x7FFFFFFF || (M + gm::BM - 1) / gm::BM > 65535)
+        return W4A16_ERR_UNSUPPORTED;
+    plan_gemm(M, N, K, sms, opt, pl);
+    if (pl->splits > 1) return W4A16_ERR_UNSUPPORTED;   // split-K reduction not built yet
+    return W4A16_OK;
 }
 
 // ------------------------------------------------------------------ launches
@@ -306,6 +335,38 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
+int launch_gemm(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void *stream, bool pdl) {
+    CUtensorMap tm_x, tm_w;
+    // x: [M, K] BF16, boxes of 64 columns x 128 rows, 128-byte swizzle (K-major operand layout)
+    int rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, 64, gm::BM,
+                       CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    // codes: [N, K/8] uint32, one group (16 words) x 128 rows
+    rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16, gm::BN,
+                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+    gm::Params kp;
+    kp.scales = static_cast<const uint16_t *>(p.scales);
+    kp.biases = static_cast<const uint16_t *>(p.biases);
+    kp.y = static_cast<uint16_t *>(p.y);
+    kp.M = static_cast<int>(p.M);
+    kp.N = static_cast<int>(p.N);
+    kp.G = static_cast<int>(p.K / 128);
+    kp.splits = pl.splits;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid_x, pl.grid_y, pl.grid_z);
+    cfg.blockDim = dim3(pl.block, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_w, kp);
+    return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+}
+
 int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     int rc = validate(p);
     if (rc) return rc;
@@ -338,7 +399,7 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
         if (rc) return rc;
         return launch_matvec(d, ws, p, pl, stream, pdl, pdl && static_weights);
     }
-    return W4A16_ERR_UNSUPPORTED;
+    return launch_gemm(d, p, pl, stream, pdl);
 }
 
 // ------------------------------------------------------------------ allocation-free matvec
