@@ -58,13 +58,19 @@ constexpr int kOffBar = kOffSB + kSBSlots * kSBBytes;
 constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kBStages + 2 * kSBSlots + 2 * kAccBufs;
 constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM address, + alignment slack
 static_assert(kOffB % 1024 == 0 && kBAtom % 1024 == 0 && kXAtom % 1024 == 0, "swizzled tiles need 1 KB alignment");
+// Split-K partial tile [BM][kPartStride] FP32, reusing the B stages once the main loop
+// is over; rows padded to 132 floats so that 8 threads storing 8 rows hit 8 bank groups.
+constexpr int kPartStride = BN + 4;
+constexpr int kOffPart = kOffB;
+static_assert(BM * kPartStride * 4 <= kBStages * kBBytes, "partial tile must fit in the B stages");
+constexpr int kMaxSplits = 8;           // portable cluster size
 
 struct Params {
     const uint16_t *scales;   // bf16 [N, G]
     const uint16_t *biases;   // bf16 [N, G]
     uint16_t *y;              // bf16 [M, N]
     int M, N, G;
-    int splits;               // K splits (gridDim.z)
+    int splits;               // K splits (gridDim.x, the cluster size)
 };
 
 __device__ __forceinline__ uint32_t bf16x2_plus128(uint32_t v, uint32_t v4, uint32_t sel) {
@@ -87,7 +93,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int tile_n = blockIdx.x, tile_m = blockIdx.y, split = blockIdx.z;
+    const int split = blockIdx.x, tile_n = blockIdx.y, tile_m = blockIdx.z;   // splits of a tile: one cluster
     const int G = p.G;
     const int g0 = static_cast<int>(static_cast<long long>(split) * G / p.splits);
     const int g1 = static_cast<int>(static_cast<long long>(split + 1) * G / p.splits);
@@ -263,8 +269,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&sb_empty[ss]);
             }
         }
-        // store: row m, columns n0 .. n0 + 63
-        if (m < p.M) {
+        if (p.splits > 1) {
+            // split-K: publish this CTA's partial tile; the cluster reduces it below
+            float *part = reinterpret_cast<float *>(smem + kOffPart);
+            const int rl = quarter * 32 + lane;
+#pragma unroll
+            for (int c = 0; c < 16; ++c)
+                *reinterpret_cast<float4 *>(part + rl * kPartStride + 64 * half + 4 * c) =
+                    make_float4(acc[4 * c], acc[4 * c + 1], acc[4 * c + 2], acc[4 * c + 3]);
+        } else if (m < p.M) {
+            // store: row m, columns n0 .. n0 + 63
             const long long n0 = static_cast<long long>(tile_n) * BN + 64 * half;
             uint16_t *dst = p.y + static_cast<long long>(m) * p.N + n0;
 #pragma unroll
@@ -291,6 +305,41 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp == kWarpMma) {
         tc_fence_after();
         tmem_dealloc(tmem_base, kTmemCols);
+    }
+
+    if (p.splits > 1) {
+        // Split-K reduction over the cluster (the S splits of this tile): CTA rank r sums
+        // rows [r*R, (r+1)*R) of the S partial tiles, in rank order, through distributed
+        // shared memory, and writes them to y.
+        cluster_sync_all();
+        const int S = p.splits;
+        const uint32_t rank = cluster_ctarank();
+        const int rows_per = (BM + S - 1) / S;
+        const int r_lo = static_cast<int>(rank) * rows_per;
+        const int r_hi = min(BM, r_lo + rows_per);
+        const uint32_t part0 = smem_u32(smem + kOffPart);
+        for (int item = threadIdx.x; item < (r_hi - r_lo) * (BN / 4); item += kThreads) {
+            const int rl = r_lo + item / (BN / 4), c4 = item % (BN / 4);
+            const uint32_t off = part0 + (rl * kPartStride + 4 * c4) * 4;
+            float4 v = ld_dsmem_f4(dsmem_addr(off, 0));
+            for (int sp = 1; sp < S; ++sp) {
+                const float4 w = ld_dsmem_f4(dsmem_addr(off, sp));
+                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+            }
+            const long long mrow = static_cast<long long>(tile_m) * BM + rl;
+            const long long n = static_cast<long long>(tile_n) * BN + 4 * c4;
+            if (mrow < p.M) {
+                uint16_t *dst = p.y + mrow * p.N + n;
+                if (n + 4 <= p.N && (p.N & 3) == 0) {
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));
+                } else {
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+                    for (int j = 0; j < 4; ++j)
+                        if (n + j < p.N) dst[j] = __bfloat16_as_ushort(__float2bfloat16_rn(vv[j]));
+                }
+            }
+        }
+        cluster_sync_all();   // no CTA leaves while another still reads its shared memory
     }
 }
 

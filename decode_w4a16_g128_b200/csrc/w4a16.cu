@@ -188,7 +188,8 @@ int choose_path(int64_t M, const w4a16_options *opt, int *path) {
 
 int validate_options(const w4a16_options *opt) {
     if (!opt) return W4A16_OK;
-    if (opt->splits < 0 || opt->splits > 16 || opt->workers < 0 || opt->sm_count < 0) return W4A16_ERR_INVALID_ARG;
+    if (opt->splits < 0 || opt->splits > gm::kMaxSplits || opt->workers < 0 || opt->sm_count < 0)
+        return W4A16_ERR_INVALID_ARG;
     if (opt->flags & ~(W4A16_FLAG_NO_PDL | W4A16_FLAG_STATIC_WEIGHTS)) return W4A16_ERR_INVALID_ARG;
     return W4A16_OK;
 }
@@ -243,17 +244,25 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
     (void)sms;
     const int64_t G = K / 128;
     const int64_t tm = (M + gm::BM - 1) / gm::BM, tn = (N + gm::BN - 1) / gm::BN;
-    int64_t splits = (opt && opt->splits > 0) ? opt->splits : 1;
-    splits = std::max<int64_t>(1, std::min<int64_t>(splits, G));
+    int64_t splits = 1;
+    if (opt && opt->splits > 0) {
+        splits = opt->splits;
+    } else {
+        // split K only when the tiles leave SMs idle; the splits of a tile form a cluster
+        const int64_t tiles = tm * tn;
+        if (tiles < sms) splits = std::min<int64_t>(sms / tiles, gm::kMaxSplits);
+        splits = std::min<int64_t>(splits, G / 2 > 0 ? G / 2 : 1);   // at least two groups per split
+    }
+    splits = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(splits, G), gm::kMaxSplits));
     std::memset(pl, 0, sizeof(*pl));
     pl->path = W4A16_PATH_GEMM;
     pl->splits = static_cast<int32_t>(splits);
-    pl->grid_x = static_cast<int32_t>(tn);
-    pl->grid_y = static_cast<int32_t>(tm);
-    pl->grid_z = static_cast<int32_t>(splits);
+    pl->grid_x = static_cast<int32_t>(splits);   // the splits of a tile are one cluster
+    pl->grid_y = static_cast<int32_t>(tn);
+    pl->grid_z = static_cast<int32_t>(tm);
     pl->block = gm::kThreads;
     pl->smem_bytes = gm::kSmemBytes;
-    pl->cluster = 1;
+    pl->cluster = static_cast<int32_t>(splits);
     pl->tiles = tm * tn;
     pl->units = tm * tn * G;
     pl->workspace_bytes = 0;
@@ -267,10 +276,8 @@ int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a
         plan_matvec(M, N, K, sms, opt, pl);
         return W4A16_OK;
     }
-    if (N >= (int64_t(1) << 31) / 1 || (N + gm::BN - 1) / gm::BN > 0x7FFFFFFF || (M + gm::BM - 1) / gm::BM > 65535)
-        return W4A16_ERR_UNSUPPORTED;
+    if ((N + gm::BN - 1) / gm::BN > 65535 || (M + gm::BM - 1) / gm::BM > 65535) return W4A16_ERR_UNSUPPORTED;
     plan_gemm(M, N, K, sms, opt, pl);
-    if (pl->splits > 1) return W4A16_ERR_UNSUPPORTED;   // split-K reduction not built yet
     return W4A16_OK;
 }
 
@@ -358,11 +365,20 @@ int launch_gemm(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void
     cfg.blockDim = dim3(pl.block, 1, 1);
     cfg.dynamicSmemBytes = pl.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    attr[na].id = cudaLaunchAttributeClusterDimension;
+    attr[na].val.clusterDim.x = pl.cluster;
+    attr[na].val.clusterDim.y = 1;
+    attr[na].val.clusterDim.z = 1;
+    ++na;
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
+    cfg.numAttrs = na;
     cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_w, kp);
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }

@@ -92,7 +92,7 @@ int w4a16_matmul_last_rows(const void *x, const uint32_t *wq, const void *scales
 /* Options for the explicit entry points; zero-initialised means "automatic". */
 typedef struct w4a16_options {
     int32_t path;      /* enum w4a16_path                                                  */
-    int32_t splits;    /* GEMM: K splits (1..16), each a contiguous run of 128-groups; 0 = auto */
+    int32_t splits;    /* GEMM: K splits (1..8), each a contiguous run of 128-groups; 0 = auto */
     int32_t workers;   /* matvec: persistent CTAs sharing the (row-tile x group) units; 0 = auto */
     int32_t sm_count;  /* w4a16_plan only: SM count to plan for; 0 = query the current device   */
     int32_t flags;     /* W4A16_FLAG_* bits                                                 */

@@ -119,3 +119,27 @@ def test_logits_to_keep_lm_head():
     ref_last = oracle_y(prob, np.array([63]))
     assert_close(bits(last), ref_last, "last row")
     assert_close(bits(full)[63:64], ref_last, "row 63 of all rows")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 5, 8])
+@pytest.mark.parametrize("M,N,K", [(128, 1000, 1024), (300, 257, 1024), (17, 130, 768)])
+def test_split_k_integer_bit_exact(splits, M, N, K):
+    prob = synth.make_integer_problem(M, N, K)
+    got = run(prob, path=w4.PATH_GEMM, splits=splits)
+    assert np.array_equal(got, oracle_y(prob)), f"splits={splits} M={M} N={N} K={K}"
+
+
+@pytest.mark.parametrize("splits", [2, 4, 7, 8])
+def test_split_k_down_proj(splits):
+    prob = synth.make_problem(128, 2560, 9728, outliers=True)
+    assert_close(run(prob, path=w4.PATH_GEMM, splits=splits), oracle_y(prob), f"down_proj splits={splits}")
+
+
+def test_split_k_deterministic():
+    prob = synth.make_problem(128, 1024, 2560)
+    d = to_device(prob)
+    assert w4.w4a16_plan(128, 1024, 2560)["splits"] > 1
+    outs = [bits(w4.w4a16_matmul(d["x"], d["wq"], d["scales"], d["biases"])) for _ in range(10)]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+    assert_close(outs[0], oracle_y(prob))
