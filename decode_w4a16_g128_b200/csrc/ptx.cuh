@@ -68,6 +68,34 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Same test, but a thread whose phase is not complete yet may be suspended by
+// the hardware for up to `hint_ns` (it resumes as soon as the phase completes),
+// so waiting warps do not take issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity, uint32_t hint_ns) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+        : "memory");
+    return ok != 0;
+}
+
+// Non-blocking test of a phase (never suspends).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
 __device__ __forceinline__ bool status_set() {
     return *static_cast<volatile int *>(&g_status) != 0;
 }
@@ -81,7 +109,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t spin = 1;; ++spin) {
-        if (mbar_try_wait(bar, parity)) return true;
+        if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
         if ((spin & 63u) == 0) {
             if (give_up_on_status && status_set()) return false;
             if (globaltimer() - t0 > kWaitTimeoutNs) {
@@ -132,6 +160,13 @@ __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t *bar) {
                  : "memory");
 }
 
+// Order this thread's earlier generic-proxy accesses of global memory (e.g. an
+// acquire load that made another CTA's writes visible) before its later
+// async-proxy accesses (bulk copies reading that memory).
+__device__ __forceinline__ void fence_proxy_async_global() {
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
 // ------------------------------------------------------------------ loads
 
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
@@ -139,6 +174,17 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "r"(addr));
+    return v;
+}
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint4 v) {
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+                 : "memory");
+}
+
+__device__ __forceinline__ float2 lds_f2(uint32_t addr) {
+    float2 v;
+    asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(addr));
     return v;
 }
 
@@ -161,7 +207,7 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 // so OR-ing a code into the low mantissa bits gives 128 + code exactly.
 __device__ __forceinline__ uint32_t codes_to_bf16x2_plus128(uint32_t v) {
     uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xEA;" : "=r"(r) : "r"(v), "r"(0x000F000Fu), "r"(0x43004300u));
+    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(v));
     return r;
 }
 
@@ -205,6 +251,20 @@ __device__ __forceinline__ int atomic_add_acq_rel_gpu(int *addr, int v) {
     int old;
     asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], %2;" : "=r"(old) : "l"(addr), "r"(v) : "memory");
     return old;
+}
+
+// Release-add at GPU scope (no return value): every write that happens-before
+// it, including other threads' writes ordered through a CTA barrier or an
+// mbarrier phase this thread observed, is visible to a GPU-scope acquire that
+// reads the new value.
+__device__ __forceinline__ void red_release_gpu_add(int *addr, int v) {
+    asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(addr), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ int ld_acquire_gpu(const int *addr) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(addr) : "memory");
+    return v;
 }
 
 // ------------------------------------------------------------------ named barriers

@@ -25,12 +25,11 @@ namespace {
 
 constexpr int kVersion = 100;          // 0.1.0
 constexpr int kMinTickets = 1 << 16;   // ticket slots allocated up front (grows on demand)
-// Shared memory a matvec CTA may use so that a CTA of the next launch in the
-// stream fits beside it on the same SM (programmatic dependent launch).
-constexpr long long kMatvecPairBudget = 112 * 1024;
-constexpr long long kMatvecSoloBudget = 220 * 1024;
+// Shared memory of a matvec CTA: one CTA per SM, most of the SM's shared
+// memory, so that the copy ring is deep enough to cover HBM latency.
+constexpr long long kMatvecBudget = 220 * 1024;
 constexpr int kMatvecMaxStages = 10;
-constexpr int kMatvecMinStages = 3;
+constexpr int kMatvecMinStages = 4;
 
 std::atomic<int> g_last_cuda_error{0};
 
@@ -49,7 +48,7 @@ struct DeviceInfo {
 struct Workspace {
     float *partials = nullptr;
     size_t partial_floats = 0;
-    int *tickets = nullptr;
+    int *tickets = nullptr;     // per-tile flags of the matvec fix-up, zero between launches
     int64_t ticket_count = 0;
 };
 
@@ -76,7 +75,7 @@ int device_setup(int dev, DeviceInfo **out) {
             if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
             d.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
             e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     int(kMatvecSoloBudget));
+                                     int(kMatvecBudget));
             if (e == cudaSuccess)   // one carveout for every launch: no reconfiguration between them
                 e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e == cudaSuccess)
@@ -197,19 +196,19 @@ int validate_options(const w4a16_options *opt) {
 // ------------------------------------------------------------------ planning
 
 // Ring depth and scale/bias slab slots of the matvec for G groups: two slab
-// slots and as many stages as fit the pair budget; one slot when two do not
-// leave kMatvecMinStages; a solo-CTA budget, then no slab, for very long K.
+// slots (the next tile's scales load while this one's are in use) and as many
+// stages as fit; one slot, then none (scales read from global memory), when
+// two slots would leave fewer than kMatvecMinStages stages.
 void matvec_smem_plan(int64_t G, int *stages, int *slots, long long *bytes) {
-    auto fit = [&](long long budget, int nslots) {
+    auto fit = [&](int nslots) {
         for (int st = kMatvecMaxStages; st >= kMatvecMinStages; --st)
-            if (mv::smem_bytes(st, nslots, G) <= budget) return st;
+            if (mv::smem_bytes(st, nslots, G) <= kMatvecBudget) return st;
         return 0;
     };
     int st = 0, sl = 0;
-    if ((st = fit(kMatvecPairBudget, 2))) sl = 2;
-    else if ((st = fit(kMatvecPairBudget, 1))) sl = 1;
-    else if ((st = fit(kMatvecSoloBudget, 1))) sl = 1;
-    else { st = fit(kMatvecPairBudget, 0); sl = 0; }
+    for (sl = 2; sl >= 0; --sl)
+        if ((st = fit(sl))) break;
+    if (sl < 0) sl = 0;
     *stages = st;
     *slots = sl;
     *bytes = mv::smem_bytes(st, sl, G);
@@ -235,7 +234,7 @@ void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
     pl->cluster = 1;
     pl->tiles = tiles;
     pl->units = units;
-    pl->workspace_bytes = int64_t(workers) * 2 * mv::kRows * 8 * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
+    pl->workspace_bytes = int64_t(workers) * mv::kPartialFloats * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
 }
 
 // Tensor-core GEMM: 128 x 128 output tiles; K split into `splits` contiguous runs
@@ -307,7 +306,7 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     int rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2,
                        16 * mv::kGroupsPerStage, mv::kRows, CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
-    // x viewed as [M, K/2] pairs of BF16: box of 264 BF16 (132 pairs) x M rows
+    // x viewed as [M, K/2] pairs of BF16: box of 256 BF16 (128 pairs) x M rows
     rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.x, p.K / 2, p.M, p.K * 2, mv::kXCols / 2,
                    static_cast<uint32_t>(p.M), CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
@@ -316,7 +315,7 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     kp.biases = static_cast<const uint16_t *>(p.biases);
     kp.y = static_cast<uint16_t *>(p.y);
     kp.partials = ws->partials;
-    kp.tickets = ws->tickets;
+    kp.flags = ws->tickets;
     kp.M = static_cast<int>(p.M);
     kp.N = static_cast<int>(p.N);
     kp.G = static_cast<int>(p.K / 128);
@@ -326,7 +325,7 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     long long smem = 0;
     matvec_smem_plan(kp.G, &kp.stages, &kp.slab_slots, &smem);
     kp.slab_array_bytes = static_cast<int>(mv::slab_array_bytes(kp.G));
-    kp.flags = static_weights ? mv::kFlagStaticWeights : 0;
+    kp.opts = static_weights ? mv::kFlagStaticWeights : 0;
 
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid_x, 1, 1);
@@ -411,7 +410,7 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     const bool static_weights = opt && (opt->flags & W4A16_FLAG_STATIC_WEIGHTS);
     if (pl.path == W4A16_PATH_MATVEC) {
         Workspace *ws = nullptr;
-        rc = workspace_get(dev, stream, size_t(pl.grid_x) * 2 * mv::kRows * 8, pl.tiles, &ws);
+        rc = workspace_get(dev, stream, size_t(pl.grid_x) * mv::kPartialFloats, pl.tiles, &ws);
         if (rc) return rc;
         return launch_matvec(d, ws, p, pl, stream, pdl, pdl && static_weights);
     }
@@ -420,11 +419,14 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
 
 // ------------------------------------------------------------------ allocation-free matvec
 
-// Scratch of w4a16_matvec_noalloc: FP32 partials of up to kNoAllocWorkers CTAs,
-// then one ticket per 128-row tile for up to W4A16_NOALLOC_MAX_N rows.
+// Scratch of w4a16_matvec_noalloc: a region for the FP32 partials of up to
+// kNoAllocWorkers CTAs (8 KB each, of which the kernel uses the first
+// kPartialFloats), then one flag per 128 rows for up to W4A16_NOALLOC_MAX_N rows.
 constexpr int kNoAllocWorkers = 160;
-constexpr size_t kNoAllocPartialBytes = size_t(kNoAllocWorkers) * 2 * mv::kRows * 8 * sizeof(float);
-constexpr int64_t kNoAllocTiles = W4A16_NOALLOC_MAX_N / mv::kRows;
+constexpr size_t kNoAllocPartialBytes = size_t(kNoAllocWorkers) * 8192;
+static_assert(mv::kPartialFloats * sizeof(float) <= 8192, "partial slot exceeds its scratch share");
+constexpr int64_t kNoAllocTiles = W4A16_NOALLOC_MAX_N / 128;   // flag slots: at least one per tile
+static_assert(mv::kRows >= 128, "flag region sized for tiles of 128 rows or more");
 static_assert(kNoAllocPartialBytes + kNoAllocTiles * sizeof(int) == W4A16_NOALLOC_SCRATCH_BYTES,
               "header and scratch layout disagree");
 static __device__ __align__(256) unsigned char g_noalloc_scratch[W4A16_NOALLOC_SCRATCH_BYTES];
@@ -468,7 +470,7 @@ int noalloc_matvec(const Problem &p, void *stream) {
     ws.partial_floats = kNoAllocPartialBytes / sizeof(float);
     ws.tickets = reinterpret_cast<int *>(it->second + kNoAllocPartialBytes);
     ws.ticket_count = kNoAllocTiles;
-    // the tickets of this call must start at zero whatever an earlier call left behind
+    // the flags of this call must start at zero whatever an earlier call left behind
     cudaError_t e = cudaMemsetAsync(ws.tickets, 0, size_t(pl.tiles) * sizeof(int), static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
     return launch_matvec(d, &ws, p, pl, stream, /*pdl=*/true, /*static_weights=*/false);

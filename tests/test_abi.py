@@ -105,8 +105,8 @@ def test_dispatch_rule():
                                  (151936, 2560), (1000, 256), (8, 128)])
 def test_matvec_plan(N, K):
     pl = w4.w4a16_plan(1, N, K, sm_count=148)
-    rows = 16 * (pl["block"] // 32 - 1)
-    assert pl["tiles"] == -(-N // rows)
+    assert pl["block"] == 672   # producer warp, 4 x-preparation warps, 16 consumer warps
+    assert pl["tiles"] == -(-N // 256)   # 16 consumer warps x 16 rows
     assert pl["units"] == pl["tiles"] * (K // 128)
     assert 1 <= pl["grid_x"] <= min(148, pl["units"])
     assert pl["smem_bytes"] <= 227 * 1024
