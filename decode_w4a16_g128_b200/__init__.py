@@ -5,7 +5,7 @@ device pointers and the current CUDA stream to the C ABI declared in
 ``include/w4a16.h`` and turns a non-zero status into ``W4A16Error``.  All
 arithmetic runs in the library's CUDA kernels; there is no fallback, and
 importing this package fails loudly when the shared library has not been
-built (``python -m decode_w4a16_g128_b200.build``).
+built (``python decode_w4a16_g128_b200/build.py``).
 
 Tensors: ``x`` bf16 [M, K]; ``wq`` int32/uint32 [N, K/8] (eight 4-bit codes
 per word, low nibble first); ``scales``/``biases`` bf16 [N, K/128]; the result
@@ -57,7 +57,7 @@ class PlanInfo(ctypes.Structure):
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIBRARY_PATH):
         raise ImportError(f"{LIBRARY_PATH} is missing: build it with "
-                          "`python -m decode_w4a16_g128_b200.build` (needs nvcc)")
+                          "`python decode_w4a16_g128_b200/build.py` (needs nvcc)")
     lib = ctypes.CDLL(LIBRARY_PATH)
     p, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
     lib.w4a16_matmul.argtypes = [p, p, p, p, p, i64, i64, i64, p]
