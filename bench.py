@@ -50,7 +50,7 @@ METRIC = "W4A16 matmul TFLOP/s & GB/s on 1 B200 vs roofline fraction (M=1..2048)
 DECODE_M = (1, 2, 4, 8)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 KERNEL_SOURCES = ("decode_w4a16_g128_b200/csrc/matvec.cuh", "decode_w4a16_g128_b200/csrc/ptx.cuh")
-TRAFFIC_FILE = os.path.join(ROOT, "profiles", "matvec_decode_traffic.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "matvec_decode_traffic.txt")
 
 
 def algo_bytes(M, N, K):
@@ -59,6 +59,20 @@ def algo_bytes(M, N, K):
 
 def decode_calls():
     return [(M, name, K, N) for M in DECODE_M for (name, K, N) in synth.QWEN3_4B_PROJECTIONS]
+
+
+PREFILL_SETS = (
+    ("prefill_m128", "M=128 over the seven Qwen3-4B projections (aligned tiles)",
+     [(128, name, K, N, 0) for (name, K, N) in synth.QWEN3_4B_PROJECTIONS]),
+    ("partial_long_k", "M in {129,509} x N in {1000,4096} x K in {2560,9728}, x with 1% outliers x20",
+     [(M, f"M{M}_N{N}_K{K}", K, N, 0) for M in (129, 509) for N in (1000, 4096) for K in (2560, 9728)]),
+    ("prefill_m2048", "M=2048 over the seven Qwen3-4B projections",
+     [(2048, name, K, N, 0) for (name, K, N) in synth.QWEN3_4B_PROJECTIONS]),
+    ("lm_head_last_row", "lm_head 2560->151936 on the last of 2048 rows (logits_to_keep=1)",
+     [(2048, "lm_head", 2560, 151936, 1)]),
+    ("lm_head_all_rows", "lm_head 2560->151936 on all 2048 rows",
+     [(2048, "lm_head", 2560, 151936, 0)]),
+)
 
 
 def peaks():
@@ -85,12 +99,13 @@ def recorded_traffic():
     """Per-launch DRAM bytes from the committed ncu capture, if it matches this kernel."""
     try:
         with open(TRAFFIC_FILE) as f:
-            d = json.load(f)
-    except (OSError, ValueError):
+            d = dict(line.split(":", 1) for line in f if ":" in line and not line.startswith("#"))
+        d = {k.strip(): v.strip() for k, v in d.items()}
+        if d.get("kernel_sha") != kernel_hash():
+            return None
+        return int(d["dram_bytes_per_launch"])
+    except (OSError, ValueError, KeyError):
         return None
-    if d.get("kernel_sha") != kernel_hash():
-        return None
-    return d.get("dram_bytes_per_launch")
 
 
 # ---------------------------------------------------------------- clocks
@@ -257,11 +272,14 @@ def run_ours(args, world, rank, local):
 
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
+    if args.mode == "profile" and args.case:
+        return profile_case(args, device, torch.cuda.Stream(device))
     if world > 1:
         init_group(world, "nccl")
     pk = peaks()
 
     weights, xs = make_host_inputs()
+    weights_cache = {(name, K, N): weights[name] for (name, K, N) in synth.QWEN3_4B_PROJECTIONS}
     calls = decode_calls()
     nsets = 2
 
@@ -379,12 +397,22 @@ def run_ours(args, world, rank, local):
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         import oracle
-        nb, t = cpu_sample(weights, xs, 1.0)
+        nb, t, reps = 0, 0.0, 0
+        while t < args.cpu_seconds or reps == 0:   # whole decode steps until the time bound is reached
+            b_, t_ = cpu_sample(weights, xs, 1.0)
+            nb, t, reps = nb + b_, t + t_, reps + 1
         cpu = {"value": round(nb / t / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
-               "sample": "one full decode step (all 28 calls) through the C oracle, OpenMP over outputs"}
+               "sample": f"{reps} full decode steps (all 28 calls each, {t:.1f} s) through the C oracle, "
+                         "OpenMP over outputs"}
 
     if args.detail and rank == 0:
         detail(args, sets[0], calls, stream, pk)
+
+    prefill = None
+    if not args.no_prefill:
+        del sets, graphs
+        torch.cuda.empty_cache()
+        prefill = prefill_section(device, stream, pk, weights_cache)
 
     if rank == 0:
         line = {
@@ -403,11 +431,120 @@ def run_ours(args, world, rank, local):
             "gpu_launches": launches * args.steps,
             "clocks": clocks,
         }
+        if prefill is not None:
+            m2048 = prefill["prefill_m2048"]
+            line["roofline_gemm"] = {
+                "bound": "tensor", "achieved": m2048["tflops"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                "frac": m2048["frac"], "traffic": None, "peak_source": pk["source"] + " (burst)",
+                "kernel": "w4a16::gm::gemm_kernel", "workload": "M=2048, seven Qwen3-4B projections"}
+            line["prefill"] = prefill
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
-        del graphs
         dist.destroy_process_group()
+    return 0
+
+
+def time_calls(make_copy, launch, n_copies, reps, stream):
+    """Mean device time (us) of one call: a CUDA graph of `reps` back-to-back calls
+    rotating over `n_copies` distinct input sets, replayed 3 times after a warm-up."""
+    import torch
+    copies = [make_copy(i) for i in range(n_copies)]
+    with torch.cuda.stream(stream):
+        for c in copies:
+            launch(c)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(reps):
+            launch(copies[i % n_copies])
+    with torch.cuda.stream(stream):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(3):
+            g.replay()
+        e1.record(stream)
+    torch.cuda.synchronize()
+    us = e0.elapsed_time(e1) * 1e3 / (3 * reps)
+    del g, copies
+    return us
+
+
+def prefill_section(device, stream, pk, weights_cache):
+    """Time every M > 8 configuration (and the last-row vocabulary projection)."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    out = {}
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    flop_peak = pk["bf16_tflops"]
+    for key, desc, calls in PREFILL_SETS:
+        rows, tot_flops, tot_us, tot_bytes = [], 0, 0.0, 0
+        for (M, name, K, N, keep) in calls:
+            if (name, K, N) not in weights_cache:
+                weights_cache[(name, K, N)] = synth.make_weights(synth.shape_rng(0, N, K, seed=0), N, K)
+            wq, sc, bi = weights_cache[(name, K, N)]
+            outliers = key == "partial_long_k"
+            x_host = synth.make_x(synth.shape_rng(M, N, K, seed=1), M, K, outliers=outliers)
+            Mo = M if keep == 0 else keep
+            wbytes = algo_bytes(M, N, K)
+            n_copies = int(max(2, min(16, math.ceil(2.2 * l2 / wbytes))))
+            base = (torch.from_numpy(x_host.view(np.int16)).to(device).view(torch.bfloat16),
+                    torch.from_numpy(wq.view(np.int32)).to(device),
+                    torch.from_numpy(sc.view(np.int16)).to(device).view(torch.bfloat16),
+                    torch.from_numpy(bi.view(np.int16)).to(device).view(torch.bfloat16))
+
+            def make_copy(i, base=base, Mo=Mo, N=N):
+                t = base if i == 0 else tuple(a.clone() for a in base)
+                return t + (torch.empty((Mo, N), dtype=torch.bfloat16, device=device),)
+
+            def launch(c, keep=keep):
+                x, q, s_, b_, y = c
+                if keep:
+                    w4.w4a16_matmul_last_rows(x, q, s_, b_, keep, y=y)
+                else:
+                    w4.w4a16_matmul(x, q, s_, b_, y=y)
+
+            flops = 2 * Mo * N * K
+            reps = int(max(4, min(64, 2e9 / max(flops, 1))))
+            us = time_calls(make_copy, launch, n_copies, reps, stream)
+            del base
+            b = algo_bytes(Mo, N, K)
+            rows.append({"M": Mo, "proj": name, "N": N, "K": K, "us": round(us, 3),
+                         "tflops": round(flops / us / 1e6, 2), "gbs": round(b / us / 1e3, 1),
+                         "frac_tensor": round(flops / us / 1e6 / flop_peak, 4),
+                         "frac_hbm": round(b / us / 1e3 / pk["hbm_gbs"], 4)})
+            tot_flops += flops
+            tot_us += us
+            tot_bytes += b
+        agg_tf = tot_flops / tot_us / 1e6
+        agg_gb = tot_bytes / tot_us / 1e3
+        bound = "hbm" if key == "lm_head_last_row" else "tensor"
+        out[key] = {"workload": desc, "us": round(tot_us, 3), "tflops": round(agg_tf, 2),
+                    "gbs": round(agg_gb, 1), "bound": bound,
+                    "frac": round(agg_gb / pk["hbm_gbs"] if bound == "hbm" else agg_tf / flop_peak, 4),
+                    "calls": rows}
+        torch.cuda.empty_cache()
+    return out
+
+
+def profile_case(args, device, stream):
+    """Three eager calls of one M x N x K problem (for an ncu capture of one kernel)."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    M, N, K = (int(v) for v in args.case.split(","))
+    prob = synth.make_problem(M, N, K)
+    d = [torch.from_numpy(prob[k].view(np.int16 if prob[k].dtype == np.uint16 else np.int32)).to(device)
+         for k in ("x", "wq", "scales", "biases")]
+    x, wq, sc, bi = d[0].view(torch.bfloat16), d[1], d[2].view(torch.bfloat16), d[3].view(torch.bfloat16)
+    y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            w4.w4a16_matmul(x, wq, sc, bi, y=y)
+    torch.cuda.synchronize()
+    if w4.w4a16_device_status(stream) != w4.OK:
+        raise RuntimeError("device status not ok")
     return 0
 
 
@@ -459,6 +596,9 @@ def main():
     ap.add_argument("--mode", choices=("bench", "profile"), default="bench")
     ap.add_argument("--detail", action="store_true", help="also time every call on its own")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-prefill", action="store_true", help="skip the M > 8 measurements")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0, help="time bound of the CPU baseline sample")
+    ap.add_argument("--case", default="", help="profile mode: one problem 'M,N,K' (three eager calls)")
     ap.add_argument("--ref-fraction", type=float, default=0.125,
                     help="reference arm: fraction of each call's output columns per step")
     args = ap.parse_args()

@@ -42,6 +42,7 @@ struct DeviceInfo {
     bool ready = false;
     int status = W4A16_OK;
     int sms = 0;
+    bool gemm_ok = false;     // the GEMM's register split fits its launch allocation
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
 };
 
@@ -50,6 +51,8 @@ struct Workspace {
     size_t partial_floats = 0;
     int *tickets = nullptr;     // per-tile flags of the matvec fix-up, zero between launches
     int64_t ticket_count = 0;
+    uint16_t *xs = nullptr;     // GEMM bias-step operands: x group sums [M, Kx], then coefficients [N, Kx]
+    size_t xs_elems = 0;
 };
 
 std::mutex g_mu;
@@ -74,6 +77,14 @@ int device_setup(int dev, DeviceInfo **out) {
             e = cudaGetDriverEntryPointByVersion("cuTensorMapEncodeTiled", &fn, 12000, cudaEnableDefault, &q);
             if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn) return cuda_fail(e);
             d.encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+            // The GEMM's warpgroups rebalance registers with setmaxnreg; a split larger than
+            // the allocation the kernel is launched with would never be granted, so the GEMM
+            // path is refused (W4A16_ERR_UNSUPPORTED) unless it fits.
+            cudaFuncAttributes fa{};
+            e = cudaFuncGetAttributes(&fa, gm::gemm_kernel);
+            if (e != cudaSuccess) return cuda_fail(e);
+            d.gemm_ok = fa.numRegs * gm::kThreads >=
+                        128 * (gm::kRegsCtl + 2 * gm::kRegsDeq + 2 * gm::kRegsEpi);
             e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      int(kMatvecBudget));
             if (e == cudaSuccess)   // one carveout for every launch: no reconfiguration between them
@@ -129,6 +140,29 @@ int workspace_get(int dev, void *stream, size_t partial_floats, int64_t tickets,
             if (e != cudaSuccess) return cuda_fail(e);
             w.ticket_count = count;
         }
+    }
+    *out = &w;
+    return W4A16_OK;
+}
+
+// The GEMM's bias-step operand buffer of (device, stream), grown to at least `elems` BF16 values.
+int workspace_xs(int dev, void *stream, size_t elems, Workspace **out) {
+    Workspace &w = g_workspaces[{dev, stream}];
+    if (w.xs_elems < elems) {
+        cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+        cudaError_t e = cudaStreamIsCapturing(static_cast<cudaStream_t>(stream), &cap);
+        if (e != cudaSuccess) return cuda_fail(e);
+        if (cap != cudaStreamCaptureStatusNone) return W4A16_ERR_UNSUPPORTED;
+        e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));   // the old buffer may be in use
+        if (e != cudaSuccess) return cuda_fail(e);
+        cudaFree(w.xs);
+        w.xs = nullptr;
+        w.xs_elems = 0;
+        if (cudaMalloc(&w.xs, elems * sizeof(uint16_t)) != cudaSuccess) {
+            cudaGetLastError();
+            return W4A16_ERR_NO_MEMORY;
+        }
+        w.xs_elems = elems;
     }
     *out = &w;
     return W4A16_OK;
@@ -264,7 +298,7 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
     pl->cluster = static_cast<int32_t>(splits);
     pl->tiles = tm * tn;
     pl->units = tm * tn * G;
-    pl->workspace_bytes = 0;
+    pl->workspace_bytes = (M + N) * gm::xs_cols(static_cast<int>(G)) * 2;   // bias-step operands
 }
 
 int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a16_plan_info *pl) {
@@ -341,44 +375,67 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
-int launch_gemm(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void *stream, bool pdl) {
-    CUtensorMap tm_x, tm_w;
-    // x: [M, K] BF16, boxes of 64 columns x 128 rows, 128-byte swizzle (K-major operand layout)
+int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan_info &pl, void *stream,
+                bool pdl, bool static_weights) {
+    const int G = static_cast<int>(p.K / 128);
+    const int Kx = gm::xs_cols(G);
+    CUtensorMap tm_x, tm_xs;
+    // x: [M, K] BF16, boxes of 64 columns x 128 rows, 128-byte swizzle (K-major B operand)
     int rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, 64, gm::BM,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
-    // codes: [N, K/8] uint32, one group (16 words) x 128 rows
-    rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16, gm::BN,
-                   CU_TENSOR_MAP_SWIZZLE_NONE);
+    // group sums of x: [M, Kx] BF16, same boxes
+    rc = encode_2d(d, &tm_xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws->xs, Kx, p.M, uint64_t(Kx) * 2, 64, gm::BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
+    cudaLaunchAttribute pdl_attr;
+    pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    pdl_attr.val.programmaticStreamSerializationAllowed = 1;
+
+    // 1. bias-step operands: group sums of x and the matching weight coefficients
+    uint16_t *bc = ws->xs + size_t(p.M) * Kx;
+    {
+        const long long items = (p.M + p.N) * G;
+        const long long blocks = std::min<long long>((items + 255) / 256, static_cast<long long>(d->sms) * 8);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(blocks, 1)), 1, 1);
+        cfg.blockDim = dim3(256, 1, 1);
+        cfg.stream = static_cast<cudaStream_t>(stream);
+        cfg.attrs = &pdl_attr;
+        cfg.numAttrs = pdl ? 1 : 0;
+        cudaError_t e = cudaLaunchKernelEx(&cfg, gm::prep_kernel, static_cast<const uint16_t *>(p.x),
+                                           static_cast<const uint16_t *>(p.scales),
+                                           static_cast<const uint16_t *>(p.biases), ws->xs, bc,
+                                           static_cast<int>(p.M), static_cast<int>(p.N), G, Kx);
+        if (e != cudaSuccess) return cuda_fail(e);
+    }
+    // 2. the GEMM (programmatic dependent launch on the group sums)
     gm::Params kp;
+    kp.wq = p.wq;
     kp.scales = static_cast<const uint16_t *>(p.scales);
     kp.biases = static_cast<const uint16_t *>(p.biases);
+    kp.bc = bc;
     kp.y = static_cast<uint16_t *>(p.y);
     kp.M = static_cast<int>(p.M);
     kp.N = static_cast<int>(p.N);
-    kp.G = static_cast<int>(p.K / 128);
+    kp.G = G;
+    kp.Kx = Kx;
     kp.splits = pl.splits;
+    kp.static_weights = static_weights ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid_x, pl.grid_y, pl.grid_z);
     cfg.blockDim = dim3(pl.block, 1, 1);
     cfg.dynamicSmemBytes = pl.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
     cudaLaunchAttribute attr[2];
-    int na = 0;
-    attr[na].id = cudaLaunchAttributeClusterDimension;
-    attr[na].val.clusterDim.x = pl.cluster;
-    attr[na].val.clusterDim.y = 1;
-    attr[na].val.clusterDim.z = 1;
-    ++na;
-    if (pdl) {
-        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-        attr[na].val.programmaticStreamSerializationAllowed = 1;
-        ++na;
-    }
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = pl.cluster;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    attr[1] = pdl_attr;
     cfg.attrs = attr;
-    cfg.numAttrs = na;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_w, kp);
+    cfg.numAttrs = pdl ? 2 : 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_xs, kp);
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
@@ -414,7 +471,11 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
         if (rc) return rc;
         return launch_matvec(d, ws, p, pl, stream, pdl, pdl && static_weights);
     }
-    return launch_gemm(d, p, pl, stream, pdl);
+    if (!d->gemm_ok) return W4A16_ERR_UNSUPPORTED;
+    Workspace *ws = nullptr;
+    rc = workspace_xs(dev, stream, size_t(p.M + p.N) * gm::xs_cols(static_cast<int>(p.K / 128)), &ws);
+    if (rc) return rc;
+    return launch_gemm(d, ws, p, pl, stream, pdl, pdl && static_weights);
 }
 
 // ------------------------------------------------------------------ allocation-free matvec
@@ -560,6 +621,7 @@ void w4a16_release(void) {
         cudaDeviceSynchronize();
         cudaFree(kv.second.partials);
         cudaFree(kv.second.tickets);
+        cudaFree(kv.second.xs);
     }
     g_workspaces.clear();
     cudaSetDevice(cur);
