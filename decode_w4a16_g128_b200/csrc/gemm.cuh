@@ -30,10 +30,18 @@
 // padded with zeros to Kx = 128 ceil(6 G / 128) columns.  The GEMM runs Kx / 128
 // extra "bias steps" (A = a 128-column block of Bc, B = the same block of Xs),
 // spread round-robin over the K splits and added with scale 1.
-// One CTA computes a BN x BM = 128 x 128 tile of y^T over a contiguous range of
-// 128-groups (all of K, or one split of a cluster).  Warp roles (20 warps):
+// Two CTAs on two SMs (a CTA pair, tcgen05 cta_group::2) compute a 256 x 128 tile of
+// y^T: each CTA dequantises its own 128 weight rows into its own tensor memory and
+// stages 64 of the 128 x rows; the pair leader issues M = 256 MMAs that read both
+// halves of each operand, so every x byte loaded from L2 serves 256 weight rows.
+// Both CTAs' TMA bytes and dequantisation arrivals land on the leader's barriers;
+// the leader's commits are multicast to both CTAs.  A cluster holds the S K-splits
+// of a tile as S pairs (cluster rank = 2 split + pair rank).  Warp roles (20 warps
+// per CTA):
 //   warp 0 (one thread)  TMA producer of the x / Xs stages (bias steps first)
-//   warp 1 (one thread)  MMA issuer (and TMEM allocation)
+//   warp 2 (one thread)  TMA producer of the packed codes (64-byte swizzle)
+//   warps 1, 3 (one thread each)  MMA issuers in the pair leader, even / odd steps
+//                        (warp 1 also allocates tensor memory, in both CTAs)
 //   warps 4-11           dequantisation: warp w owns lanes 32 (w % 4) .. +31 and
 //                        the column half (w - 4) / 4 of each A buffer
 //   warps 12-19          epilogue: lanes 32 (w % 4) .. +31, x rows 64 ((w - 12) / 4) .. +63
@@ -46,13 +54,15 @@
 namespace w4a16 {
 namespace gm {
 
-constexpr int BN = 128;                 // weight rows of a tile: MMA M, TMEM lanes
+constexpr int BN = 128;                 // weight rows of a CTA: its half of the pair MMA's M = 256
+constexpr int kPairRows = 2 * BN;       // weight rows of a CTA pair (one output tile)
 constexpr int BM = 128;                 // x rows of a tile: MMA N, accumulator columns
-constexpr int kXStages = 4;
+constexpr int kXRows = BM / 2;          // x rows staged by each CTA of the pair (its half of B)
+constexpr int kXStages = 8;
 constexpr int kABufs = 3;
 constexpr int kDBufs = 2;
-constexpr int kXAtom = BM * 128;        // 64 k of 128 x rows, 128-byte swizzle: 16 KB
-constexpr int kXBytes = 2 * kXAtom;     // one group: 32 KB
+constexpr int kXAtom = kXRows * 128;    // 64 k of 64 x rows, 128-byte swizzle: 8 KB
+constexpr int kXBytes = 2 * kXAtom;     // one group of this CTA's x rows: 16 KB
 constexpr int kACols = 64;              // 128 BF16 values of a row
 constexpr int kACol0 = kDBufs * BM;     // A buffers follow the accumulators
 constexpr int kTmemCols = 512;
@@ -61,7 +71,7 @@ static_assert(kACol0 + kABufs * kACols <= kTmemCols, "tensor memory budget");
 constexpr int kWarpTma = 0, kWarpMma = 1, kWarpDeq = 4, kDeqWarps = 8, kWarpEpi = 12, kEpiWarps = 8;
 constexpr int kThreads = (kWarpEpi + kEpiWarps) * 32;   // 640
 constexpr int kLaunchRegs = 96;                         // per thread at launch (65536 / 640, rounded to 8)
-constexpr int kRegsCtl = 32, kRegsDeq = 72, kRegsEpi = 152;
+constexpr int kRegsCtl = 56, kRegsDeq = 56, kRegsEpi = 152;
 // Registers are exchanged within each SM sub-partition, which holds one warp of every
 // warpgroup: a warpgroup that grows must never race one that has not yet shrunk.  The
 // epilogue grows at the start (the others shrink unconditionally first) and shrinks at
@@ -71,18 +81,31 @@ static_assert(128 * (kRegsCtl + 2 * kRegsDeq + 2 * kRegsEpi) <= kThreads * kLaun
               "register split exceeds the launch allocation");
 
 constexpr int kBiasCoef = 6;            // bias-step entries per group
-constexpr int kOffBar = kXStages * kXBytes;
+constexpr int kWStages = 4;             // packed codes ring
+constexpr int kWBytes = BN * 64;        // one group's codes of this CTA's 128 rows: 8 KB
+constexpr int kOffW = kXStages * kXBytes;
+constexpr int kOffBar = kOffW + kWStages * kWBytes;
 // Barriers, indexed by step i: ready[i % kXStages] (x or Xs landed + every dequantisation
 // warp stored A), done[i % kXStages] (the step's MMAs completed: frees its x stage, its A
 // buffer and fills its accumulator), d_empty[i % kDBufs] (the epilogue read the accumulator).
 // No waiter can be a whole ring behind the phase it waits for (each role is at most
-// kXStages - 1 steps ahead of the next), so the parities never alias.
-constexpr int kNumBars = 2 * kXStages + kDBufs;
+// kXStages - 1 steps ahead of the next), so the parities never alias.  Per group j of
+// codes: w_full[j % kWStages] (TMA landed), w_empty[j % kWStages] (dequantisation read it).
+constexpr int kNumBars = 2 * kXStages + kDBufs + 2 * kWStages;
 static_assert(kABufs < kXStages && kDBufs < kXStages, "one done ring serves every buffer");
-constexpr int kSmemBytes = kOffBar + kNumBars * 8 + 16 + 1024;   // + TMEM address, + alignment slack
-// Split-K partial tile, [BM x rows][BN weight rows] FP32, in the x stages once the loop is over.
+static_assert(kNumBars * 8 + 16 <= 512, "barrier area");
+// The scales of this CTA's 128 rows, [128][G] BF16, staged once per CTA after the barriers.
+constexpr int kOffScales = kOffBar + 512;
+constexpr int kMaxGroups = 256;         // K <= 32768 on the GEMM path
+__host__ __device__ constexpr int smem_bytes(int G) { return kOffScales + 256 * G + 1024; }   // + alignment slack
+static_assert(smem_bytes(kMaxGroups) <= 232448, "shared memory budget");
+constexpr uint32_t kBarScales = 2;      // named barrier: the epilogue's staged scales are complete
+constexpr int kWarpCodes = 2;           // TMA producer of the packed codes
+constexpr int kWarpMma2 = 3;            // second MMA issuer (odd steps)
+static_assert(kDBufs == 2, "each of the two MMA issuers owns one accumulator");
+// Split-K partial of a CTA, [BM x rows][BN weight rows] FP32, in the x stages once the loop is over.
 static_assert(BM * BN * 4 <= kXStages * kXBytes, "partial tile must fit in the x stages");
-constexpr int kMaxSplits = 8;           // portable cluster size
+constexpr int kMaxSplits = 4;           // a cluster holds 2 x splits CTAs: at most 8 (portable size)
 
 __host__ __device__ constexpr int bias_steps(int G) { return (kBiasCoef * G + 127) / 128; }
 __host__ __device__ constexpr int xs_cols(int G) { return 128 * bias_steps(G); }
@@ -166,16 +189,23 @@ __device__ __forceinline__ uint32_t bf16x2_plus128(uint32_t v, uint32_t v4, uint
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xs,
-                const Params p) {
+                const __grid_constant__ CUtensorMap tm_w, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
     uint64_t *ready = bars, *done = ready + kXStages, *d_empty = done + kXStages;
+    uint64_t *w_full = d_empty + kDBufs, *w_empty = w_full + kWStages;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
+    uint16_t *sc_smem = reinterpret_cast<uint16_t *>(smem + kOffScales);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int split = blockIdx.x, tile_n = blockIdx.y, tile_m = blockIdx.z;   // splits of a tile: one cluster
+    const uint32_t rank = cluster_ctarank();               // 2 split + pair rank
+    const int pair_rank = static_cast<int>(rank & 1u);
+    const uint32_t leader = rank & ~1u;
+    const bool is_leader = pair_rank == 0;
+    const int split = static_cast<int>(rank >> 1);
+    const int tile_n = blockIdx.y, tile_m = blockIdx.z;
     const int G = p.G;
     const int g0 = static_cast<int>(static_cast<long long>(split) * G / p.splits);
     const int g1 = static_cast<int>(static_cast<long long>(split + 1) * G / p.splits);
@@ -184,26 +214,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nbias_all = p.Kx / 128;
     const int nbs = split < nbias_all ? (nbias_all - split + p.splits - 1) / p.splits : 0;
     const int steps = nbs + ng;
+    const long long row0 = static_cast<long long>(tile_n) * kPairRows + pair_rank * BN;   // this CTA's weight rows
 
     if (threadIdx.x == 0) {
         pdl_launch_dependents();
-        for (int i = 0; i < kXStages; ++i) { mbar_init(&ready[i], 1 + kDeqWarps); mbar_init(&done[i], 1); }
-        for (int i = 0; i < kDBufs; ++i) mbar_init(&d_empty[i], kEpiWarps);
+        for (int i = 0; i < kXStages; ++i) { mbar_init(&ready[i], 1 + 2 * kDeqWarps); mbar_init(&done[i], 1); }
+        for (int i = 0; i < kDBufs; ++i) mbar_init(&d_empty[i], 2 * kEpiWarps);
+        for (int i = 0; i < kWStages; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], kDeqWarps); }
         fence_mbar_init();
     }
-    if (warp == kWarpMma) {   // the whole warp allocates tensor memory
-        tmem_alloc(tmem_slot, kTmemCols);
-        tmem_relinquish();
+    if (warp == kWarpMma) {   // one warp of each CTA of the pair allocates the pair's tensor memory
+        tmem_alloc_pair(tmem_slot, kTmemCols);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
-    __syncthreads();
+    cluster_sync_all();   // barriers initialised and tensor memory allocated in every CTA of the cluster
     tc_fence_after();
     const uint32_t tmem_base = *tmem_slot;
+    // the leader's barriers, as shared::cluster addresses
+    const uint32_t ready_l = dsmem_addr(smem_u32(ready), leader);
+    const uint32_t d_empty_l = dsmem_addr(smem_u32(d_empty), leader);
 
     if (warp < kWarpDeq) {
         regs_shrink<kRegsCtl>();
         if (warp == kWarpTma && lane == 0) {
-            // -------------------------------------------------------- TMA producer
+            // -------------------------------------------------------- TMA producer (both CTAs)
             prefetch_tmap(&tm_x);
             prefetch_tmap(&tm_xs);
             pdl_wait();   // x (and the group sums) come from the preceding kernels
@@ -211,20 +246,39 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (; i < steps; ++i) {
                 const int s = i % kXStages;
                 if (i >= kXStages && !mbar_wait(&done[s], ((i / kXStages) - 1) & 1)) break;   // stage free
-                mbar_arrive_expect_tx(&ready[s], kXBytes);
+                if (is_leader) mbar_arrive_expect_tx(&ready[s], 2 * kXBytes);   // both halves
                 uint8_t *dst = smem + s * kXBytes;
                 const CUtensorMap *map = i < nbs ? &tm_xs : &tm_x;
                 const int col = i < nbs ? (split + i * p.splits) * 128 : (g0 + i - nbs) * 128;
-                tma_load_2d(dst, map, &ready[s], col, tile_m * BM);
-                tma_load_2d(dst + kXAtom, map, &ready[s], col + 64, tile_m * BM);
+                const int xrow = tile_m * BM + pair_rank * kXRows;
+                tma_load_2d_pair(dst, map, ready_l + 8 * s, col, xrow);
+                tma_load_2d_pair(dst + kXAtom, map, ready_l + 8 * s, col + 64, xrow);
             }
             // leave no copy in flight: the last stages' MMAs (which consumed them) completed
             for (int j = max(0, i - kXStages); j < i; ++j)
                 mbar_wait(&done[j % kXStages], (j / kXStages) & 1, false);
-        } else if (warp == kWarpMma && lane == 0) {
-            // -------------------------------------------------------- MMA issuer
-            constexpr uint32_t idesc = umma_idesc_bf16(BN, BM);
-            for (int i = 0; i < steps; ++i) {
+        } else if (warp == kWarpCodes && lane == 0) {
+            // -------------------------------------------------------- TMA producer of the codes (both CTAs)
+            prefetch_tmap(&tm_w);
+            if (!p.static_weights) pdl_wait();
+            int j = 0;
+            for (; j < ng; ++j) {
+                const int s = j % kWStages;
+                if (j >= kWStages && !mbar_wait(&w_empty[s], ((j / kWStages) - 1) & 1)) break;
+                mbar_arrive_expect_tx(&w_full[s], kWBytes);
+                tma_load_2d(smem + kOffW + s * kWBytes, &tm_w, &w_full[s], (g0 + j) * 16, static_cast<int>(row0));
+            }
+            for (int q = max(0, j - kWStages); q < j; ++q)   // leave no copy in flight
+                mbar_wait(&w_full[q % kWStages], (q / kWStages) & 1, false);
+        } else if ((warp == kWarpMma || warp == kWarpMma2) && lane == 0 && is_leader) {
+            // -------------------------------------------------------- MMA issuers (pair leader)
+            // The tensor pipe takes about one instruction ahead, so every barrier operation of
+            // an issuing thread leaves it idle for its latency.  Two issuers take alternate
+            // steps (so each always fills the same accumulator): one waits for its step's
+            // inputs while the other's MMAs run.
+            constexpr uint32_t idesc = umma_idesc_bf16(kPairRows, BM);
+            const uint16_t mask = static_cast<uint16_t>(3u << leader);
+            for (int i = (warp == kWarpMma ? 0 : 1); i < steps; i += 2) {
                 const int xs = i % kXStages, ab = i % kABufs, db = i % kDBufs;
                 if (!mbar_wait(&ready[xs], (i / kXStages) & 1)) break;
                 if (i >= kDBufs && !mbar_wait(&d_empty[db], ((i / kDBufs) - 1) & 1)) break;
@@ -235,9 +289,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t bd = umma_desc_sw128(b0 + (kk >> 2) * kXAtom + (kk & 3) * 32);
-                    umma_bf16_ts(d, a + 8 * kk, bd, idesc, kk > 0);
+                    umma_bf16_ts_pair(d, a + 8 * kk, bd, idesc, kk > 0);
                 }
-                umma_commit(&done[xs]);
+                umma_commit_pair(&done[xs], mask);
             }
         }
         __syncwarp();
@@ -245,87 +299,91 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_grow<kLaunchRegs>();             // back to the launch allocation for the common tail
     } else if (warp < kWarpEpi) {
         regs_shrink<kRegsDeq>();
-        // ------------------------------------------------------------ dequantisation
+        // ------------------------------------------------------------ dequantisation (both CTAs)
         const int quarter = warp & 3, half = (warp - kWarpDeq) >> 2;
-        const long long row = static_cast<long long>(tile_n) * BN + quarter * 32 + lane;   // weight row n
+        const long long row = row0 + quarter * 32 + lane;   // weight row n
         const bool row_ok = row < p.N;
-        const uint4 *codes = reinterpret_cast<const uint4 *>(p.wq + (row_ok ? row : 0) * (static_cast<long long>(G) * 16));
+        const int rl = quarter * 32 + lane;                  // row within the CTA's codes tile
+        const uint32_t sw = static_cast<uint32_t>((rl >> 1) & 3);   // 64-byte swizzle of that row
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kACol0 + half * 32;
-        // codes of step i (words 8 half .. 8 half + 7 of its group), fetched two steps ahead;
-        // bias steps carry zeros through the ring
-        auto fetch = [&](int i, uint4 &lo, uint4 &hi) {
-            if (row_ok && i >= nbs && i < steps) {
-                const int g = g0 + i - nbs;
-                lo = ldg_nc_v4(codes + g * 4 + 2 * half);
-                hi = ldg_nc_v4(codes + g * 4 + 2 * half + 1);
-            } else {
-                lo = hi = make_uint4(0, 0, 0, 0);
-            }
-        };
-        if (!p.static_weights) pdl_wait();
-        uint4 c0, c1, n0, n1, f0, f1;
-        fetch(0, c0, c1);
-        fetch(1, n0, n1);
         pdl_wait();   // the bias-step coefficients come from the preparation kernel
         const uint4 *bcrow = reinterpret_cast<const uint4 *>(p.bc + (row_ok ? row : 0) * static_cast<long long>(p.Kx));
         for (int i = 0; i < steps; ++i) {
             const int ab = i % kABufs;
-            fetch(i + 2, f0, f1);
-            if (i >= kABufs && !mbar_wait(&done[(i - kABufs) % kXStages], ((i - kABufs) / kXStages) & 1)) break;
-            tc_fence_after();   // the tensor cores' reads of this buffer precede the stores below
             uint32_t r[32];
             if (i >= nbs) {
+                // chunks 2 half, 2 half + 1 (words 8 half .. 8 half + 7) of this row's codes
+                const int j = i - nbs, ws = j % kWStages;
+                if (!mbar_wait(&w_full[ws], (j / kWStages) & 1)) break;
+                const uint32_t wrow = smem_u32(smem + kOffW + ws * kWBytes) + rl * 64;
+                const uint4 c0 = lds128(wrow + (((2u * half) ^ sw) << 4));
+                const uint4 c1 = lds128(wrow + (((2u * half + 1u) ^ sw) << 4));
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&w_empty[ws]);   // the codes are in registers
+                if (i >= kABufs && !mbar_wait(&done[(i - kABufs) % kXStages], ((i - kABufs) / kXStages) & 1)) break;
+                tc_fence_after();   // the tensor cores' reads of this buffer precede the stores below
                 const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {   // word j: k = 8 j .. 8 j + 7 -> columns 4 j .. 4 j + 3
-                    const uint32_t v = w[j], v4 = v >> 4;
-                    r[4 * j + 0] = bf16x2_plus128(v, v4, 0x0400u);
-                    r[4 * j + 1] = bf16x2_plus128(v, v4, 0x0501u);
-                    r[4 * j + 2] = bf16x2_plus128(v, v4, 0x0602u);
-                    r[4 * j + 3] = bf16x2_plus128(v, v4, 0x0703u);
+                for (int jj = 0; jj < 8; ++jj) {   // word jj: k = 8 jj .. 8 jj + 7 -> columns 4 jj .. 4 jj + 3
+                    const uint32_t v = w[jj], v4 = v >> 4;
+                    r[4 * jj + 0] = bf16x2_plus128(v, v4, 0x0400u);
+                    r[4 * jj + 1] = bf16x2_plus128(v, v4, 0x0501u);
+                    r[4 * jj + 2] = bf16x2_plus128(v, v4, 0x0602u);
+                    r[4 * jj + 3] = bf16x2_plus128(v, v4, 0x0703u);
                 }
             } else {   // 64 coefficients of this column half (bias steps are few: loaded here)
                 const int t = split + i * p.splits;
+                uint4 v[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const uint4 v = row_ok ? ldg_nc_v4(bcrow + t * 16 + half * 8 + j) : make_uint4(0, 0, 0, 0);
-                    r[4 * j + 0] = v.x;
-                    r[4 * j + 1] = v.y;
-                    r[4 * j + 2] = v.z;
-                    r[4 * j + 3] = v.w;
+                for (int jj = 0; jj < 8; ++jj)
+                    v[jj] = row_ok ? ldg_nc_v4(bcrow + t * 16 + half * 8 + jj) : make_uint4(0, 0, 0, 0);
+                if (i >= kABufs && !mbar_wait(&done[(i - kABufs) % kXStages], ((i - kABufs) / kXStages) & 1)) break;
+                tc_fence_after();
+#pragma unroll
+                for (int jj = 0; jj < 8; ++jj) {
+                    r[4 * jj + 0] = v[jj].x;
+                    r[4 * jj + 1] = v[jj].y;
+                    r[4 * jj + 2] = v[jj].z;
+                    r[4 * jj + 3] = v[jj].w;
                 }
             }
-            c0 = n0; c1 = n1; n0 = f0; n1 = f1;
             tmem_st32(taddr + ab * kACols, r);
             tmem_st_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&ready[i % kXStages]);
+            if (lane == 0) mbar_arrive_cluster(ready_l + 8 * (i % kXStages));
         }
         named_bar_sync(kBarRegs, kThreads);
         regs_grow<kLaunchRegs>();
     } else {
         regs_grow<kRegsEpi>();
-        // ------------------------------------------------------------ epilogue
+        // ------------------------------------------------------------ epilogue (both CTAs)
         const int quarter = warp & 3, half = (warp - kWarpEpi) >> 2;
-        const int nl = quarter * 32 + lane;                         // weight row within the tile
-        const long long row = static_cast<long long>(tile_n) * BN + nl;
+        const int nl = quarter * 32 + lane;                         // weight row within the CTA
+        const long long row = row0 + nl;
         const bool row_ok = row < p.N;
-        const uint16_t *srow = p.scales + (row_ok ? row : 0) * G;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * 64;
         if (!p.static_weights) pdl_wait();   // scales are weights
+        {
+            // stage the scales of this CTA's rows ([128][G] BF16, contiguous in global memory)
+            // with coalesced loads; no load of this warp stays in flight across its arrivals
+            const int t = threadIdx.x - kWarpEpi * 32;
+            const long long rows = min(static_cast<long long>(BN), max(0ll, p.N - row0));
+            const long long elems = rows * G;
+            const uint16_t *src = p.scales + row0 * G;
+            const long long vec = (elems * 2) / 16;
+            for (long long v = t; v < vec; v += kEpiWarps * 32)
+                reinterpret_cast<uint4 *>(sc_smem)[v] = ldg_nc_v4(reinterpret_cast<const uint4 *>(src) + v);
+            for (long long e = vec * 8 + t; e < elems; e += kEpiWarps * 32) sc_smem[e] = __ldg(src + e);
+        }
+        named_bar_sync(kBarScales, kEpiWarps * 32);
+        const uint16_t *srow = sc_smem + nl * G;
         float acc[64];
 #pragma unroll
         for (int j = 0; j < 64; ++j) acc[j] = 0.f;
-        // scale of step i (1 for bias steps), fetched four steps ahead
-        auto scale_of = [&](int i) {
-            return (row_ok && i >= nbs && i < steps) ? bf16_to_f32(__ldg(srow + g0 + i - nbs)) : 1.f;
-        };
-        float q0 = scale_of(0), q1 = scale_of(1), q2 = scale_of(2), q3 = scale_of(3);
         for (int i = 0; i < steps; ++i) {
             const int db = i % kDBufs;
-            const float sc = q0;
-            q0 = q1; q1 = q2; q2 = q3; q3 = scale_of(i + 4);
+            const float sc = (row_ok && i >= nbs) ? bf16_to_f32(srow[g0 + i - nbs]) : 1.f;
             if (!mbar_wait(&done[i % kXStages], (i / kXStages) & 1)) break;
             tc_fence_after();
             uint32_t r0[32], r1[32];
@@ -334,7 +392,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld_wait();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&d_empty[db]);
+            if (lane == 0) mbar_arrive_cluster(d_empty_l + 8 * db);
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 acc[j] = fmaf(sc, __uint_as_float(r0[j]), acc[j]);
@@ -362,32 +420,33 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncthreads();
     if (warp == kWarpMma) {
         tc_fence_after();
-        tmem_dealloc(tmem_base, kTmemCols);
+        tmem_dealloc_pair(tmem_base, kTmemCols);
     }
 
+    // Every CTA of the cluster is done with its peers' barriers and shared memory only
+    // after this barrier: none leaves while another may still signal or read it.
+    cluster_sync_all();
     if (p.splits > 1) {
-        // Split-K reduction over the cluster (the S splits of this tile): CTA rank r sums
-        // x rows [r*R, (r+1)*R) of the S partial tiles, in rank order, through distributed
-        // shared memory, and writes them to y.  The epilogue warps do the work.
-        cluster_sync_all();
+        // Split-K reduction over the S pairs of the cluster: the CTAs with this pair rank
+        // hold the S partials of the same 128 weight rows; the one of split r sums x rows
+        // [r*R, (r+1)*R) of them, in split order, through distributed shared memory.
         if (warp >= kWarpEpi) {
             const int S = p.splits;
-            const uint32_t rank = cluster_ctarank();
             const int rows_per = (BM + S - 1) / S;
-            const int r_lo = static_cast<int>(rank) * rows_per;
+            const int r_lo = split * rows_per;
             const int r_hi = min(BM, r_lo + rows_per);
             const uint32_t part0 = smem_u32(smem);
             const int t = threadIdx.x - kWarpEpi * 32;
             for (int item = t; item < (r_hi - r_lo) * (BN / 4); item += kEpiWarps * 32) {
                 const int ml = r_lo + item / (BN / 4), c4 = item % (BN / 4);
                 const uint32_t off = part0 + (ml * BN + 4 * c4) * 4;
-                float4 v = ld_dsmem_f4(dsmem_addr(off, 0));
+                float4 v = ld_dsmem_f4(dsmem_addr(off, static_cast<uint32_t>(pair_rank)));
                 for (int sp = 1; sp < S; ++sp) {
-                    const float4 w = ld_dsmem_f4(dsmem_addr(off, sp));
+                    const float4 w = ld_dsmem_f4(dsmem_addr(off, static_cast<uint32_t>(2 * sp + pair_rank)));
                     v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
                 }
                 const long long mrow = static_cast<long long>(tile_m) * BM + ml;
-                const long long n = static_cast<long long>(tile_n) * BN + 4 * c4;
+                const long long n = row0 + 4 * c4;
                 if (mrow < p.M) {
                     uint16_t *dst = p.y + mrow * p.N + n;
                     if (n + 4 <= p.N && (p.N & 3) == 0) {

@@ -90,7 +90,8 @@ int device_setup(int dev, DeviceInfo **out) {
             if (e == cudaSuccess)   // one carveout for every launch: no reconfiguration between them
                 e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, gm::kSmemBytes);
+                e = cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         gm::smem_bytes(gm::kMaxGroups));
             if (e != cudaSuccess) return cuda_fail(e);
         }
         d.ready = true;
@@ -271,31 +272,32 @@ void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
     pl->workspace_bytes = int64_t(workers) * mv::kPartialFloats * 4 + std::max<int64_t>(tiles, kMinTickets) * 4;
 }
 
-// Tensor-core GEMM: 128 x 128 output tiles; K split into `splits` contiguous runs
-// of 128-groups (forced by the options, else 1).
+// Tensor-core GEMM: output tiles of 256 weight rows x 128 x rows, each computed by a
+// CTA pair; K split into `splits` contiguous runs of 128-groups (forced by the
+// options, else chosen to fill the SMs); the splits of a tile form one cluster of
+// 2 x splits CTAs.
 void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, w4a16_plan_info *pl) {
-    (void)sms;
     const int64_t G = K / 128;
-    const int64_t tm = (M + gm::BM - 1) / gm::BM, tn = (N + gm::BN - 1) / gm::BN;
+    const int64_t tm = (M + gm::BM - 1) / gm::BM, tn = (N + gm::kPairRows - 1) / gm::kPairRows;
     int64_t splits = 1;
     if (opt && opt->splits > 0) {
         splits = opt->splits;
     } else {
-        // split K only when the tiles leave SMs idle; the splits of a tile form a cluster
-        const int64_t tiles = tm * tn;
-        if (tiles < sms) splits = std::min<int64_t>(sms / tiles, gm::kMaxSplits);
+        // split K only when the tile pairs leave SMs idle
+        const int64_t ctas = 2 * tm * tn;
+        if (ctas < sms) splits = std::min<int64_t>(sms / ctas, gm::kMaxSplits);
         splits = std::min<int64_t>(splits, G / 2 > 0 ? G / 2 : 1);   // at least two groups per split
     }
     splits = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(splits, G), gm::kMaxSplits));
     std::memset(pl, 0, sizeof(*pl));
     pl->path = W4A16_PATH_GEMM;
     pl->splits = static_cast<int32_t>(splits);
-    pl->grid_x = static_cast<int32_t>(splits);   // the splits of a tile are one cluster
+    pl->grid_x = static_cast<int32_t>(2 * splits);   // pairs of the splits of a tile: one cluster
     pl->grid_y = static_cast<int32_t>(tn);
     pl->grid_z = static_cast<int32_t>(tm);
     pl->block = gm::kThreads;
-    pl->smem_bytes = gm::kSmemBytes;
-    pl->cluster = static_cast<int32_t>(splits);
+    pl->smem_bytes = gm::smem_bytes(static_cast<int>(G));
+    pl->cluster = static_cast<int32_t>(2 * splits);
     pl->tiles = tm * tn;
     pl->units = tm * tn * G;
     pl->workspace_bytes = (M + N) * gm::xs_cols(static_cast<int>(G)) * 2;   // bias-step operands
@@ -309,7 +311,9 @@ int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a
         plan_matvec(M, N, K, sms, opt, pl);
         return W4A16_OK;
     }
-    if ((N + gm::BN - 1) / gm::BN > 65535 || (M + gm::BM - 1) / gm::BM > 65535) return W4A16_ERR_UNSUPPORTED;
+    if ((N + gm::kPairRows - 1) / gm::kPairRows > 65535 || (M + gm::BM - 1) / gm::BM > 65535 ||
+        K / 128 > gm::kMaxGroups)
+        return W4A16_ERR_UNSUPPORTED;
     plan_gemm(M, N, K, sms, opt, pl);
     return W4A16_OK;
 }
@@ -379,14 +383,19 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
                 bool pdl, bool static_weights) {
     const int G = static_cast<int>(p.K / 128);
     const int Kx = gm::xs_cols(G);
-    CUtensorMap tm_x, tm_xs;
-    // x: [M, K] BF16, boxes of 64 columns x 128 rows, 128-byte swizzle (K-major B operand)
-    int rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, 64, gm::BM,
+    CUtensorMap tm_x, tm_xs, tm_w;
+    // x: [M, K] BF16, boxes of 64 columns x 64 rows (one CTA's half of the x rows of a
+    // tile), 128-byte swizzle (K-major B operand)
+    int rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, 64, gm::kXRows,
                        CU_TENSOR_MAP_SWIZZLE_128B);
     if (rc) return rc;
     // group sums of x: [M, Kx] BF16, same boxes
-    rc = encode_2d(d, &tm_xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws->xs, Kx, p.M, uint64_t(Kx) * 2, 64, gm::BM,
+    rc = encode_2d(d, &tm_xs, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, ws->xs, Kx, p.M, uint64_t(Kx) * 2, 64, gm::kXRows,
                    CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    // codes: [N, K/8] uint32, boxes of one group (16 words = 64 B) x 128 rows, 64-byte swizzle
+    rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16, gm::BN,
+                   CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
     cudaLaunchAttribute pdl_attr;
     pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -435,7 +444,7 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     attr[1] = pdl_attr;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_xs, kp);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_xs, tm_w, kp);
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 

@@ -70,7 +70,8 @@ enum w4a16_path {
 /*
  * y = x . dequant(wq)^T.  Arguments as in the layout block above.
  * M == 0 or N == 0: returns W4A16_OK and launches nothing.
- * Sizes: 0 <= M, N < 2^31, 0 <= K < 2^31 with K % 128 == 0.
+ * Sizes: 0 <= M, N < 2^31, 0 <= K < 2^31 with K % 128 == 0; on the tensor-core
+ * GEMM path (M > 8, or forced) also K <= 32768, else W4A16_ERR_UNSUPPORTED.
  * Ownership: all buffers belong to the caller and must stay valid until the
  * enqueued work completes.
  */
@@ -92,7 +93,7 @@ int w4a16_matmul_last_rows(const void *x, const uint32_t *wq, const void *scales
 /* Options for the explicit entry points; zero-initialised means "automatic". */
 typedef struct w4a16_options {
     int32_t path;      /* enum w4a16_path                                                  */
-    int32_t splits;    /* GEMM: K splits (1..8), each a contiguous run of 128-groups; 0 = auto */
+    int32_t splits;    /* GEMM: K splits (1..4), each a contiguous run of 128-groups; 0 = auto */
     int32_t workers;   /* matvec: persistent CTAs sharing the (row-tile x group) units; 0 = auto */
     int32_t sm_count;  /* w4a16_plan only: SM count to plan for; 0 = query the current device   */
     int32_t flags;     /* W4A16_FLAG_* bits                                                 */
@@ -125,7 +126,7 @@ int w4a16_matmul_ex(const void *x, const uint32_t *wq, const void *scales,
 /* What a call of the given size would launch (host-side planning only). */
 typedef struct w4a16_plan_info {
     int32_t path;            /* enum w4a16_path chosen                                  */
-    int32_t splits;          /* GEMM K splits (cluster size along K); 1 for the matvec  */
+    int32_t splits;          /* GEMM K splits (a cluster holds 2 x splits CTAs); 1 for the matvec */
     int32_t grid_x, grid_y, grid_z;
     int32_t block;           /* threads per CTA                                         */
     int32_t smem_bytes;      /* dynamic shared memory per CTA                           */

@@ -90,9 +90,10 @@ def test_bad_options():
     opt = w4.make_options(path=w4.PATH_MATVEC)
     assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
                                P(A + 0x400000), 9, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_UNSUPPORTED
-    opt = w4.make_options(splits=9)
-    assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
-                               P(A + 0x400000), 2, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_INVALID_ARG
+    for splits in (5, 9):
+        opt = w4.make_options(splits=splits)
+        assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
+                                   P(A + 0x400000), 2, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_INVALID_ARG
 
 
 def test_dispatch_rule():
@@ -127,19 +128,35 @@ def test_streamk_owner_matches_brute_force():
     assert w4.w4a16_streamk_owner(10, 2, 10) == -1
 
 
-@pytest.mark.parametrize("M,N,K,expect_splits", [(128, 4096, 2560, 4), (128, 1024, 2560, 8), (128, 2560, 9728, 7),
-                                                 (128, 9728, 2560, 1), (2048, 4096, 2560, 1), (32, 64, 256, 1)])
+@pytest.mark.parametrize("M,N,K,expect_splits", [(128, 4096, 2560, 4), (128, 1024, 2560, 4), (128, 2560, 9728, 4),
+                                                 (128, 9728, 2560, 1), (2048, 4096, 2560, 1), (32, 64, 256, 1),
+                                                 (509, 4096, 9728, 1), (129, 1000, 9728, 4)])
 def test_gemm_split_plan(M, N, K, expect_splits):
-    """Split K only while the 128x128 tiles leave SMs idle; a tile's splits form one cluster."""
+    """Tiles of 256 weight rows x 128 x rows, each on a CTA pair; K is split only while
+    the pairs leave SMs idle, and a tile's splits form one cluster of 2 x splits CTAs."""
     pl = w4.w4a16_plan(M, N, K, sm_count=148)
     assert pl["path"] == w4.PATH_GEMM
-    assert pl["splits"] == expect_splits and pl["cluster"] == expect_splits
-    tiles = -(-M // 128) * -(-N // 128)
-    assert pl["grid_x"] * pl["grid_y"] * pl["grid_z"] == tiles * expect_splits
-    assert pl["splits"] <= 8 and pl["splits"] <= K // 128
+    assert pl["splits"] == expect_splits and pl["cluster"] == 2 * expect_splits
+    tiles = -(-M // 128) * -(-N // 256)
+    assert pl["tiles"] == tiles
+    assert pl["grid_x"] * pl["grid_y"] * pl["grid_z"] == 2 * tiles * expect_splits
+    assert pl["splits"] <= 4 and pl["splits"] <= K // 128
+    assert pl["cluster"] <= 8
 
 
 def test_gemm_forced_splits_plan():
-    for s in range(1, 9):
-        assert w4.w4a16_plan(300, 1000, 1024, path=w4.PATH_GEMM, splits=s, sm_count=148)["splits"] == min(s, 8)
-    assert w4.w4a16_plan(300, 1000, 256, path=w4.PATH_GEMM, splits=8, sm_count=148)["splits"] == 2   # G = 2
+    for s in range(1, 5):
+        assert w4.w4a16_plan(300, 1000, 1024, path=w4.PATH_GEMM, splits=s, sm_count=148)["splits"] == s
+    for s in range(5, 9):   # a cluster holds at most 8 CTAs: 4 pairs
+        with pytest.raises(w4.W4A16Error):
+            w4.w4a16_plan(300, 1000, 1024, path=w4.PATH_GEMM, splits=s, sm_count=148)
+    assert w4.w4a16_plan(300, 1000, 256, path=w4.PATH_GEMM, splits=4, sm_count=148)["splits"] == 2   # G = 2
+
+
+def test_gemm_k_limit():
+    """The tensor-core path stages each CTA's scales in shared memory: K <= 32768 there."""
+    assert w4.w4a16_plan(128, 1000, 32768, sm_count=148)["path"] == w4.PATH_GEMM
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_plan(128, 1000, 32768 + 128, sm_count=148)
+    assert e.value.status == w4.ERR_UNSUPPORTED
+    assert w4.w4a16_plan(8, 1000, 32768 + 128, sm_count=148)["path"] == w4.PATH_MATVEC   # no limit there
