@@ -59,7 +59,7 @@ constexpr int kPairRows = 2 * BN;       // weight rows of a CTA pair (one output
 constexpr int BM = 128;                 // x rows of a tile: MMA N, accumulator columns
 constexpr int kXRows = BM / 2;          // x rows staged by each CTA of the pair (its half of B)
 constexpr int kXStages = 8;
-constexpr int kABufs = 3;
+constexpr int kABufs = 4;
 constexpr int kDBufs = 2;
 constexpr int kXAtom = kXRows * 128;    // 64 k of 64 x rows, 128-byte swizzle: 8 KB
 constexpr int kXBytes = 2 * kXAtom;     // one group of this CTA's x rows: 16 KB
@@ -119,6 +119,7 @@ struct Params {
     int M, N, G, Kx;
     int splits;               // K splits (gridDim.x, the cluster size)
     int static_weights;       // codes, scales and biases may be read before the dependency wait
+    int tma_store;            // y rows are 16-byte multiples: tiles leave through one TMA store
 };
 
 // ------------------------------------------------------------------ preparation: bias-step operands
@@ -189,7 +190,7 @@ __device__ __forceinline__ uint32_t bf16x2_plus128(uint32_t v, uint32_t v4, uint
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xs,
-                const __grid_constant__ CUtensorMap tm_w, const Params p) {
+                const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_y, const Params p) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
@@ -241,6 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // -------------------------------------------------------- TMA producer (both CTAs)
             prefetch_tmap(&tm_x);
             prefetch_tmap(&tm_xs);
+            if (p.tma_store) prefetch_tmap(&tm_y);
             pdl_wait();   // x (and the group sums) come from the preceding kernels
             int i = 0;
             for (; i < steps; ++i) {
@@ -406,6 +408,19 @@ __global__ void __launch_bounds__(kThreads, 1)
             float *part = reinterpret_cast<float *>(smem);
 #pragma unroll
             for (int j = 0; j < 64; ++j) part[(half * 64 + j) * BN + nl] = acc[j];
+        } else if (p.tma_store) {
+            // the tile, [x row][weight row] BF16, into the (idle) x stages, then one TMA store
+            uint16_t *tile = reinterpret_cast<uint16_t *>(smem);
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                tile[(half * 64 + j) * BN + nl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+            fence_proxy_async_smem();   // the async proxy reads the tile
+            named_bar_sync(kBarScales, kEpiWarps * 32);
+            if (warp == kWarpEpi && lane == 0) {
+                tma_store_2d(&tm_y, tile, static_cast<int>(row0), tile_m * BM);
+                bulk_commit_group();
+                bulk_wait_all();   // shared memory is released, and y written, before the CTA ends
+            }
         } else if (row_ok) {
 #pragma unroll
             for (int j = 0; j < 64; ++j)

@@ -383,7 +383,7 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
                 bool pdl, bool static_weights) {
     const int G = static_cast<int>(p.K / 128);
     const int Kx = gm::xs_cols(G);
-    CUtensorMap tm_x, tm_xs, tm_w;
+    CUtensorMap tm_x, tm_xs, tm_w, tm_y;
     // x: [M, K] BF16, boxes of 64 columns x 64 rows (one CTA's half of the x rows of a
     // tile), 128-byte swizzle (K-major B operand)
     int rc = encode_2d(d, &tm_x, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.x, p.K, p.M, p.K * 2, 64, gm::kXRows,
@@ -397,6 +397,16 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16, gm::BN,
                    CU_TENSOR_MAP_SWIZZLE_64B);
     if (rc) return rc;
+    // y: [M, N] BF16, one box per CTA tile (128 weight rows = columns of y, 128 x rows); only
+    // when its rows are 16-byte multiples (TMA strides), else the kernel stores element-wise
+    const bool tma_store = (p.N * 2) % 16 == 0;
+    if (tma_store) {
+        rc = encode_2d(d, &tm_y, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, p.y, p.N, p.M, p.N * 2, gm::BN, gm::BM,
+                       CU_TENSOR_MAP_SWIZZLE_NONE);
+        if (rc) return rc;
+    } else {
+        std::memset(&tm_y, 0, sizeof(tm_y));
+    }
     cudaLaunchAttribute pdl_attr;
     pdl_attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
     pdl_attr.val.programmaticStreamSerializationAllowed = 1;
@@ -431,6 +441,7 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     kp.Kx = Kx;
     kp.splits = pl.splits;
     kp.static_weights = static_weights ? 1 : 0;
+    kp.tma_store = tma_store ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid_x, pl.grid_y, pl.grid_z);
     cfg.blockDim = dim3(pl.block, 1, 1);
@@ -444,7 +455,7 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     attr[1] = pdl_attr;
     cfg.attrs = attr;
     cfg.numAttrs = pdl ? 2 : 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_xs, tm_w, kp);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, gm::gemm_kernel, tm_x, tm_xs, tm_w, tm_y, kp);
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
