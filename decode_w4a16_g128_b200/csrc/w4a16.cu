@@ -249,6 +249,20 @@ void matvec_smem_plan(int64_t G, int *stages, int *slots, long long *bytes) {
     *bytes = mv::smem_bytes(st, sl, G);
 }
 
+// Persistent CTAs of the matvec.  A CTA holds most of an SM's shared memory, so the next
+// kernel of the stream (programmatic dependent launch) can only start streaming its
+// weights on SMs this one leaves free; and every tile split over several CTAs costs a
+// fix-up.  Measured on B200 with back-to-back calls: k/v 2560->1024 (80 units) is
+// fastest with 40 CTAs, q/o (320 units) with about 120, gate/up/down (760 units) with
+// about 128, and the 151936-row vocabulary projection with every SM.
+int64_t default_matvec_workers(int64_t units, int sms) {
+    const int64_t most = (int64_t(sms) * 82) / 100, more = (int64_t(sms) * 87) / 100;
+    if (units < 2 * most) return std::max<int64_t>(1, (units + 1) / 2);
+    if (units < 4 * int64_t(sms)) return most;
+    if (units < 16 * int64_t(sms)) return more;
+    return sms;
+}
+
 void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, w4a16_plan_info *pl) {
     (void)M;
     const int64_t G = K / 128;
@@ -257,7 +271,7 @@ void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
     matvec_smem_plan(G, &stages, &slots, &smem);
     const int64_t tiles = (N + mv::kRows - 1) / mv::kRows;
     const int64_t units = tiles * G;
-    int64_t workers = (opt && opt->workers > 0) ? opt->workers : sms;
+    int64_t workers = (opt && opt->workers > 0) ? opt->workers : default_matvec_workers(units, sms);
     workers = std::max<int64_t>(1, std::min<int64_t>(workers, units));
     std::memset(pl, 0, sizeof(*pl));
     pl->path = W4A16_PATH_MATVEC;

@@ -160,3 +160,13 @@ def test_gemm_k_limit():
         w4.w4a16_plan(128, 1000, 32768 + 128, sm_count=148)
     assert e.value.status == w4.ERR_UNSUPPORTED
     assert w4.w4a16_plan(8, 1000, 32768 + 128, sm_count=148)["path"] == w4.PATH_MATVEC   # no limit there
+
+
+@pytest.mark.parametrize("N,K,expect", [(1024, 2560, 40), (4096, 2560, 121), (2560, 4096, 121), (9728, 2560, 128),
+                                        (2560, 9728, 128), (151936, 2560, 148), (64, 256, 1)])
+def test_matvec_default_workers(N, K, expect):
+    """Persistent CTAs of the matvec: fewer than the SMs for small and mid-size weights (the
+    next call's CTAs start on the free SMs), every SM for the vocabulary projection."""
+    pl = w4.w4a16_plan(1, N, K, sm_count=148)
+    assert pl["path"] == w4.PATH_MATVEC and pl["grid_x"] == expect
+    assert w4.w4a16_plan(1, N, K, sm_count=148, workers=17)["grid_x"] == min(17, pl["units"])
