@@ -366,33 +366,61 @@ def run_ours(args, world, rank, local):
     achieved = step_bytes / (ms_step * 1e-3) / 1e9      # per GPU: bytes per launch / mean launch time
     traffic = recorded_traffic()
 
-    # end to end through the binding: H2D of this step's activations, 28 eager calls, D2H of outputs
-    host_x = [torch.from_numpy(xs[(M, name)].view(np.int16)).pin_memory() for (M, name, K, N) in calls]
-    host_y = [torch.empty((M, N), dtype=torch.int16).pin_memory() for (M, name, K, N) in calls]
-    h2d = sum(t.numel() * 2 for t in host_x)
-    d2h = sum(t.numel() * 2 for t in host_y)
+    # End to end through the C ABI with host buffers: one H2D copy of the step's activations
+    # (all 28 x, packed in one pinned buffer), the 28 calls, one D2H copy of the 28 outputs.
+    import ctypes
+    x_off, y_off, xo, yo = [], [], 0, 0
+    for (M, name, K, N) in calls:
+        x_off.append(xo)
+        y_off.append(yo)
+        xo += M * K
+        yo += M * N
+    host_x = torch.empty(xo, dtype=torch.int16).pin_memory()
+    for (M, name, K, N), off in zip(calls, x_off):
+        host_x[off:off + M * K] = torch.from_numpy(xs[(M, name)].view(np.int16).reshape(-1))
+    host_y = torch.empty(yo, dtype=torch.int16).pin_memory()
+    dev_x = torch.empty(xo, dtype=torch.int16, device=device)
+    dev_y = torch.empty(yo, dtype=torch.int16, device=device)
+    h2d, d2h = host_x.numel() * 2, host_y.numel() * 2
+    opt = w4.make_options(flags=flags)
+    P = ctypes.c_void_p
 
-    def e2e_step(entries):
-        for hx, hy, (x, wq, s, b, y) in zip(host_x, host_y, entries):
-            x.view(torch.int16).copy_(hx, non_blocking=True)
-            w4.w4a16_matmul_ex(x, wq, s, b, y=y, flags=flags)
-            hy.copy_(y.view(torch.int16), non_blocking=True)
+    def c_args(entries):
+        out = []
+        for (M, name, K, N), (x, wq, s_, b_, y), xo_, yo_ in zip(calls, entries, x_off, y_off):
+            out.append((P(dev_x.data_ptr() + 2 * xo_), P(wq.data_ptr()), P(s_.data_ptr()), P(b_.data_ptr()),
+                        P(dev_y.data_ptr() + 2 * yo_), M, N, K))
+        return out
+
+    set_args = [c_args(entries) for entries in sets]
+    fn = w4.lib.w4a16_matmul_ex
+    sp = P(stream.cuda_stream)
+    optp = ctypes.byref(opt)
+
+    def e2e_step(args):
+        dev_x.copy_(host_x, non_blocking=True)
+        for a in args:
+            rc = fn(*a, sp, optp)
+            if rc:
+                raise RuntimeError(f"w4a16_matmul_ex: {w4.status_string(rc)}")
+        host_y.copy_(dev_y, non_blocking=True)
 
     with torch.cuda.stream(stream):
         for i in range(args.warmup):
-            e2e_step(sets[i % nsets])
+            e2e_step(set_args[i % nsets])
     torch.cuda.synchronize()
     barrier(world)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     with torch.cuda.stream(stream):
         e0.record(stream)
         for i in range(args.steps):
-            e2e_step(sets[i % nsets])
+            e2e_step(set_args[i % nsets])
         e1.record(stream)
     torch.cuda.synchronize()
     barrier(world)
     e2e_ms = max_over_ranks(e0.elapsed_time(e1), world, device) / args.steps
     e2e_gbs = step_bytes * world / (e2e_ms * 1e-3) / 1e9
+    del dev_x, dev_y
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             tmem_st32(taddr + ab * kACols, r);
-            tmem_st_wait();
+            tmem_st_wait_regs(r);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(ready_l + 8 * (i % kXStages));
@@ -391,7 +391,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t r0[32], r1[32];
             tmem_ld32(taddr + db * BM, r0);
             tmem_ld32(taddr + db * BM + 32, r1);
-            tmem_ld_wait();
+            tmem_ld_wait_regs(r0);
+            tmem_ld_wait_regs(r1);   // both loads completed at the first wait; this only pins r1
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive_cluster(d_empty_l + 8 * db);
