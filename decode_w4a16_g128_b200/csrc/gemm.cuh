@@ -36,15 +36,20 @@
 // halves of each operand, so every x byte loaded from L2 serves 256 weight rows.
 // Both CTAs' TMA bytes and dequantisation arrivals land on the leader's barriers;
 // the leader's commits are multicast to both CTAs.  A cluster holds the S K-splits
-// of a tile as S pairs (cluster rank = 2 split + pair rank).  Warp roles (20 warps
-// per CTA):
+// of a tile as S pairs (cluster rank = 2 split + pair rank).  Without a K split the
+// grid is persistent (one pair per two SMs, each looping over tiles), so the next
+// tile's loads, dequantisation and MMAs overlap the previous tile's last steps and its
+// store.  Warp roles (20 warps per CTA):
 //   warp 0 (one thread)  TMA producer of the x / Xs stages (bias steps first)
-//   warp 2 (one thread)  TMA producer of the packed codes (64-byte swizzle)
-//   warps 1, 3 (one thread each)  MMA issuers in the pair leader, even / odd steps
-//                        (warp 1 also allocates tensor memory, in both CTAs)
+//   warp 1 (one thread)  MMA issuer in the pair leader (also allocates tensor memory,
+//                        in both CTAs)
+//   warp 2 (one thread)  TMA producer of the packed codes (64-byte swizzle), and of each
+//                        tile's scales (a 1-D bulk copy into one of two buffers)
+//   warp 3               idle
 //   warps 4-11           dequantisation: warp w owns lanes 32 (w % 4) .. +31 and
 //                        the column half (w - 4) / 4 of each A buffer
-//   warps 12-19          epilogue: lanes 32 (w % 4) .. +31, x rows 64 ((w - 12) / 4) .. +63
+//   warps 12-19          epilogue: lanes 32 (w % 4) .. +31, x rows 64 ((w - 12) / 4) .. +63;
+//                        a tile leaves through a staging buffer and one TMA store
 // Registers are rebalanced per warpgroup with setmaxnreg and returned to the
 // launch allocation before the common tail.  All waits are bounded.
 #pragma once
@@ -58,7 +63,7 @@ constexpr int BN = 128;                 // weight rows of a CTA: its half of the
 constexpr int kPairRows = 2 * BN;       // weight rows of a CTA pair (one output tile)
 constexpr int BM = 128;                 // x rows of a tile: MMA N, accumulator columns
 constexpr int kXRows = BM / 2;          // x rows staged by each CTA of the pair (its half of B)
-constexpr int kXStages = 8;
+constexpr int kXStages = 6;
 constexpr int kABufs = 4;
 constexpr int kDBufs = 2;
 constexpr int kXAtom = kXRows * 128;    // 64 k of 64 x rows, 128-byte swizzle: 8 KB
@@ -84,25 +89,35 @@ constexpr int kBiasCoef = 6;            // bias-step entries per group
 constexpr int kWStages = 4;             // packed codes ring
 constexpr int kWBytes = BN * 64;        // one group's codes of this CTA's 128 rows: 8 KB
 constexpr int kOffW = kXStages * kXBytes;
-constexpr int kOffBar = kOffW + kWStages * kWBytes;
+constexpr int kOffOut = kOffW + kWStages * kWBytes;   // output tile staging for the TMA store
+constexpr int kOutBytes = BM * BN * 2;                // [x row][weight row] BF16: 32 KB
+constexpr int kOffBar = kOffOut + kOutBytes;
 // Barriers, indexed by step i: ready[i % kXStages] (x or Xs landed + every dequantisation
 // warp stored A), done[i % kXStages] (the step's MMAs completed: frees its x stage, its A
 // buffer and fills its accumulator), d_empty[i % kDBufs] (the epilogue read the accumulator).
 // No waiter can be a whole ring behind the phase it waits for (each role is at most
 // kXStages - 1 steps ahead of the next), so the parities never alias.  Per group j of
 // codes: w_full[j % kWStages] (TMA landed), w_empty[j % kWStages] (dequantisation read it).
-constexpr int kNumBars = 2 * kXStages + kDBufs + 2 * kWStages;
+// Per output tile k of a CTA: sc_full[k % B] (its scales are staged), sc_empty[k % B] (the
+// epilogue is done with them), B = scale_bufs(G).  Step, group and tile indices run on
+// across the tiles of a persistent CTA.
+constexpr int kScaleBufsMax = 2;
+constexpr int kNumBars = 2 * kXStages + kDBufs + 2 * kWStages + 2 * kScaleBufsMax;
 static_assert(kABufs < kXStages && kDBufs < kXStages, "one done ring serves every buffer");
 static_assert(kNumBars * 8 + 16 <= 512, "barrier area");
-// The scales of this CTA's 128 rows, [128][G] BF16, staged once per CTA after the barriers.
+// The scales of a tile's 128 rows of this CTA, [128][G] BF16, after the barriers: two
+// buffers (the next tile's are staged while the epilogue reads this one's) up to 128
+// groups, one above.
 constexpr int kOffScales = kOffBar + 512;
 constexpr int kMaxGroups = 256;         // K <= 32768 on the GEMM path
-__host__ __device__ constexpr int smem_bytes(int G) { return kOffScales + 256 * G + 1024; }   // + alignment slack
-static_assert(smem_bytes(kMaxGroups) <= 232448, "shared memory budget");
-constexpr uint32_t kBarScales = 2;      // named barrier: the epilogue's staged scales are complete
+__host__ __device__ constexpr int scale_bufs(int G) { return G <= 128 ? 2 : 1; }
+__host__ __device__ constexpr int smem_bytes(int G) {
+    return kOffScales + scale_bufs(G) * 256 * G + 1024;   // + alignment slack
+}
+static_assert(smem_bytes(kMaxGroups) <= 232448 && smem_bytes(128) <= 232448, "shared memory budget");
+constexpr uint32_t kBarEpi = 2;         // named barrier of the epilogue warps (output staging)
 constexpr int kWarpCodes = 2;           // TMA producer of the packed codes
-constexpr int kWarpMma2 = 3;            // second MMA issuer (odd steps)
-static_assert(kDBufs == 2, "each of the two MMA issuers owns one accumulator");
+static_assert(kDBufs == 2 && (kABufs & (kABufs - 1)) == 0, "ring arithmetic of the MMA issuer");
 // Split-K partial of a CTA, [BM x rows][BN weight rows] FP32, in the x stages once the loop is over.
 static_assert(BM * BN * 4 <= kXStages * kXBytes, "partial tile must fit in the x stages");
 constexpr int kMaxSplits = 4;           // a cluster holds 2 x splits CTAs: at most 8 (portable size)
@@ -117,6 +132,8 @@ struct Params {
     const uint16_t *bc;       // bf16 [N, Kx] bias-step coefficients (from prep_kernel)
     uint16_t *y;              // bf16 [M, N]
     int M, N, G, Kx;
+    long long tiles;          // output tiles: tiles_n x ceil(M / 128)
+    int tiles_n;              // tiles along N (256 weight rows each)
     int splits;               // K splits (gridDim.x, the cluster size)
     int static_weights;       // codes, scales and biases may be read before the dependency wait
     int tma_store;            // y rows are 16-byte multiples: tiles leave through one TMA store
@@ -188,6 +205,58 @@ __device__ __forceinline__ uint32_t bf16x2_plus128(uint32_t v, uint32_t v4, uint
     return codes_to_bf16x2_plus128(prmt(v, v4, sel));
 }
 
+// 64 consecutive 32-bit columns of this thread's lane into registers (warp-collective;
+// the lane field of taddr is the warp's 32-lane quarter).  The registers are written
+// asynchronously: read them only after tmem_ld_wait64, which also pins them.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&r)[64]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x64.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, %48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%64];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+        : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_ld_wait64(uint32_t (&r)[64]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31]), "+r"(r[32]), "+r"(r[33]), "+r"(r[34]), "+r"(r[35]), "+r"(r[36]), "+r"(r[37]), "+r"(r[38]), "+r"(r[39]), "+r"(r[40]), "+r"(r[41]), "+r"(r[42]), "+r"(r[43]), "+r"(r[44]), "+r"(r[45]), "+r"(r[46]), "+r"(r[47]), "+r"(r[48]), "+r"(r[49]), "+r"(r[50]), "+r"(r[51]), "+r"(r[52]), "+r"(r[53]), "+r"(r[54]), "+r"(r[55]), "+r"(r[56]), "+r"(r[57]), "+r"(r[58]), "+r"(r[59]), "+r"(r[60]), "+r"(r[61]), "+r"(r[62]), "+r"(r[63]) :: "memory");
+}
+
+// a = s * x + a on two FP32 lanes at once (x a pair of FP32 bit patterns)
+__device__ __forceinline__ void ffma2(unsigned long long &a, unsigned long long s2, uint32_t x0, uint32_t x1) {
+    unsigned long long x;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(x) : "r"(x0), "r"(x1));
+    asm("fma.rn.f32x2 %0, %1, %2, %0;" : "+l"(a) : "l"(s2), "l"(x));
+}
+__device__ __forceinline__ unsigned long long f32x2(float lo, float hi) {
+    unsigned long long v;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(v) : "f"(lo), "f"(hi));
+    return v;
+}
+__device__ __forceinline__ float f32x2_lo(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v)); }
+__device__ __forceinline__ float f32x2_hi(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
+
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Tile t of the output: its x rows start at 128 m, this CTA's weight rows at row0.
+struct TileCoord {
+    int m;
+    long long row0;
+};
+__device__ __forceinline__ TileCoord tile_coord(long long t, int tiles_n, int pair_rank) {
+    const long long m = t / tiles_n;
+    return {static_cast<int>(m), (t - m * tiles_n) * kPairRows + pair_rank * BN};
+}
+
+// Position in a ring of N slots: slot and the parity of its current use.
+template <int N>
+struct RingPos {
+    int slot = 0;
+    uint32_t phase = 0;
+    __device__ __forceinline__ void advance() {
+        if (++slot == N) {
+            slot = 0;
+            phase ^= 1u;
+        }
+    }
+};
+
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_xs,
                 const __grid_constant__ CUtensorMap tm_w, const __grid_constant__ CUtensorMap tm_y, const Params p) {
@@ -196,8 +265,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
     uint64_t *ready = bars, *done = ready + kXStages, *d_empty = done + kXStages;
     uint64_t *w_full = d_empty + kDBufs, *w_empty = w_full + kWStages;
+    uint64_t *sc_full = w_empty + kWStages, *sc_empty = sc_full + kScaleBufsMax;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     uint16_t *sc_smem = reinterpret_cast<uint16_t *>(smem + kOffScales);
+    uint16_t *out_tile = reinterpret_cast<uint16_t *>(smem + kOffOut);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -206,7 +277,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t leader = rank & ~1u;
     const bool is_leader = pair_rank == 0;
     const int split = static_cast<int>(rank >> 1);
-    const int tile_n = blockIdx.y, tile_m = blockIdx.z;
     const int G = p.G;
     const int g0 = static_cast<int>(static_cast<long long>(split) * G / p.splits);
     const int g1 = static_cast<int>(static_cast<long long>(split + 1) * G / p.splits);
@@ -215,13 +285,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nbias_all = p.Kx / 128;
     const int nbs = split < nbias_all ? (nbias_all - split + p.splits - 1) / p.splits : 0;
     const int steps = nbs + ng;
-    const long long row0 = static_cast<long long>(tile_n) * kPairRows + pair_rank * BN;   // this CTA's weight rows
+    const int nsb = scale_bufs(G);
+    // Tile schedule.  Without a K split the grid is persistent: cluster c = blockIdx.y
+    // computes tiles c, c + gridDim.y, ... (tile t: tile_n = t % tiles_n, tile_m = t / tiles_n,
+    // so neighbouring clusters share x rows), and one tile's pipeline drains while the next
+    // one's fills.  With a K split each cluster computes the one tile (blockIdx.z, blockIdx.y),
+    // whose partials are reduced through shared memory at the end.
+    const bool persistent = p.splits == 1;
+    const long long tile0 = persistent ? static_cast<long long>(blockIdx.y)
+                                       : static_cast<long long>(blockIdx.z) * p.tiles_n + blockIdx.y;
+    const long long tstride = persistent ? static_cast<long long>(gridDim.y) : p.tiles;
+    const int ntl = tile0 < p.tiles ? static_cast<int>((p.tiles - tile0 + tstride - 1) / tstride) : 0;
+    const long long total = static_cast<long long>(ntl) * steps;   // steps of this CTA
 
     if (threadIdx.x == 0) {
         pdl_launch_dependents();
         for (int i = 0; i < kXStages; ++i) { mbar_init(&ready[i], 1 + 2 * kDeqWarps); mbar_init(&done[i], 1); }
         for (int i = 0; i < kDBufs; ++i) mbar_init(&d_empty[i], 2 * kEpiWarps);
         for (int i = 0; i < kWStages; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], kDeqWarps); }
+        for (int i = 0; i < kScaleBufsMax; ++i) { mbar_init(&sc_full[i], 1); mbar_init(&sc_empty[i], kEpiWarps); }
         fence_mbar_init();
     }
     if (warp == kWarpMma) {   // one warp of each CTA of the pair allocates the pair's tensor memory
@@ -239,61 +321,124 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (warp < kWarpDeq) {
         regs_shrink<kRegsCtl>();
         if (warp == kWarpTma && lane == 0) {
-            // -------------------------------------------------------- TMA producer (both CTAs)
+            // -------------------------------------------------------- TMA producer of x / Xs (both CTAs)
             prefetch_tmap(&tm_x);
             prefetch_tmap(&tm_xs);
             if (p.tma_store) prefetch_tmap(&tm_y);
             pdl_wait();   // x (and the group sums) come from the preceding kernels
-            int i = 0;
-            for (; i < steps; ++i) {
-                const int s = i % kXStages;
-                if (i >= kXStages && !mbar_wait(&done[s], ((i / kXStages) - 1) & 1)) break;   // stage free
-                if (is_leader) mbar_arrive_expect_tx(&ready[s], 2 * kXBytes);   // both halves
-                uint8_t *dst = smem + s * kXBytes;
-                const CUtensorMap *map = i < nbs ? &tm_xs : &tm_x;
-                const int col = i < nbs ? (split + i * p.splits) * 128 : (g0 + i - nbs) * 128;
-                const int xrow = tile_m * BM + pair_rank * kXRows;
-                tma_load_2d_pair(dst, map, ready_l + 8 * s, col, xrow);
-                tma_load_2d_pair(dst + kXAtom, map, ready_l + 8 * s, col + 64, xrow);
+            RingPos<kXStages> st;
+            long long issued = 0;
+            bool ok = true;
+            long long t = tile0;
+            for (int k = 0; k < ntl && ok; ++k, t += tstride) {
+                const int xrow = tile_coord(t, p.tiles_n, pair_rank).m * BM + pair_rank * kXRows;
+                for (int i = 0; i < steps; ++i) {
+                    // the stage is free once the MMAs of its previous step completed
+                    if (issued >= kXStages && !mbar_wait(&done[st.slot], st.phase ^ 1u)) { ok = false; break; }
+                    if (is_leader) mbar_arrive_expect_tx(&ready[st.slot], 2 * kXBytes);   // both halves
+                    uint8_t *dst = smem + st.slot * kXBytes;
+                    const CUtensorMap *map = i < nbs ? &tm_xs : &tm_x;
+                    const int col = i < nbs ? (split + i * p.splits) * 128 : (g0 + i - nbs) * 128;
+                    tma_load_2d_pair(dst, map, ready_l + 8 * st.slot, col, xrow);
+                    tma_load_2d_pair(dst + kXAtom, map, ready_l + 8 * st.slot, col + 64, xrow);
+                    ++issued;
+                    st.advance();
+                }
             }
             // leave no copy in flight: the last stages' MMAs (which consumed them) completed
-            for (int j = max(0, i - kXStages); j < i; ++j)
-                mbar_wait(&done[j % kXStages], (j / kXStages) & 1, false);
+            for (long long j = issued > kXStages ? issued - kXStages : 0; j < issued; ++j)
+                mbar_wait(&done[j % kXStages], static_cast<uint32_t>((j / kXStages) & 1), false);
         } else if (warp == kWarpCodes && lane == 0) {
-            // -------------------------------------------------------- TMA producer of the codes (both CTAs)
+            // -------------------------------------------------------- codes and scales, by TMA (both CTAs)
+            // The packed codes of each group, and after a tile's second group that tile's
+            // scales (one contiguous [rows][G] BF16 block: a 1-D bulk copy) into their buffer.
             prefetch_tmap(&tm_w);
             if (!p.static_weights) pdl_wait();
-            int j = 0;
-            for (; j < ng; ++j) {
-                const int s = j % kWStages;
-                if (j >= kWStages && !mbar_wait(&w_empty[s], ((j / kWStages) - 1) & 1)) break;
-                mbar_arrive_expect_tx(&w_full[s], kWBytes);
-                tma_load_2d(smem + kOffW + s * kWBytes, &tm_w, &w_full[s], (g0 + j) * 16, static_cast<int>(row0));
+            RingPos<kWStages> st;
+            long long issued = 0;
+            int staged = 0;   // tiles whose scales were staged
+            bool ok = true;
+            long long t = tile0;
+            for (int k = 0; k < ntl && ok; ++k, t += tstride) {
+                const long long row0 = tile_coord(t, p.tiles_n, pair_rank).row0;
+                const int stage_at = ng > 1 ? 1 : 0;
+                for (int j = 0; j < ng; ++j) {
+                    if (issued >= kWStages && !mbar_wait(&w_empty[st.slot], st.phase ^ 1u)) { ok = false; break; }
+                    mbar_arrive_expect_tx(&w_full[st.slot], kWBytes);
+                    tma_load_2d(smem + kOffW + st.slot * kWBytes, &tm_w, &w_full[st.slot], (g0 + j) * 16,
+                                static_cast<int>(row0));
+                    ++issued;
+                    st.advance();
+                    if (j == stage_at) {
+                        const int sb = nsb == 2 ? (k & 1) : 0;
+                        const uint32_t use = static_cast<uint32_t>(nsb == 2 ? (k >> 1) : k);
+                        // the epilogue is done with this buffer's previous tile
+                        if (k >= nsb && !mbar_wait(&sc_empty[sb], (use & 1u) ^ 1u)) { ok = false; break; }
+                        uint16_t *dst = sc_smem + sb * BN * G;
+                        const uint16_t *src = p.scales + row0 * G;   // 16-byte aligned: row0 is a multiple of 128
+                        // rows of this CTA inside y: none when the pair's second half lies past N
+                        const int rows = static_cast<int>(max(0ll, min(static_cast<long long>(BN), p.N - row0)));
+                        const uint32_t bytes = static_cast<uint32_t>(rows * G * 2);
+                        const uint32_t bulk = bytes & ~15u;
+                        for (uint32_t e = bulk / 2; e < bytes / 2; ++e) dst[e] = __ldg(src + e);   // ragged end
+                        mbar_arrive_expect_tx(&sc_full[sb], bulk);
+                        if (bulk) bulk_load(dst, src, bulk, &sc_full[sb]);
+                        ++staged;
+                    }
+                }
             }
-            for (int q = max(0, j - kWStages); q < j; ++q)   // leave no copy in flight
-                mbar_wait(&w_full[q % kWStages], (q / kWStages) & 1, false);
-        } else if ((warp == kWarpMma || warp == kWarpMma2) && lane == 0 && is_leader) {
-            // -------------------------------------------------------- MMA issuers (pair leader)
-            // The tensor pipe takes about one instruction ahead, so every barrier operation of
-            // an issuing thread leaves it idle for its latency.  Two issuers take alternate
-            // steps (so each always fills the same accumulator): one waits for its step's
-            // inputs while the other's MMAs run.
+            // leave no copy in flight
+            for (long long q = issued > kWStages ? issued - kWStages : 0; q < issued; ++q)
+                mbar_wait(&w_full[q % kWStages], static_cast<uint32_t>((q / kWStages) & 1), false);
+            for (int k = staged > nsb ? staged - nsb : 0; k < staged; ++k) {
+                const int sb = nsb == 2 ? (k & 1) : 0;
+                const uint32_t use = static_cast<uint32_t>(nsb == 2 ? (k >> 1) : k);
+                mbar_wait(&sc_full[sb], use & 1u, false);
+            }
+        } else if (warp == kWarpMma && lane == 0 && is_leader) {
+            // -------------------------------------------------------- MMA issuer (pair leader)
+            // One thread issues every step: with a second issuing thread on another SM
+            // sub-partition, the tensor-memory lanes of both sub-partitions were measured to
+            // receive wrong values now and then.  The tensor pipe takes about one instruction
+            // ahead, so a barrier operation between two steps would leave it idle: while the
+            // last four MMAs of step g run, the thread tests (without blocking) whether step
+            // g+1's inputs are in, and if so starts it with no wait.  The MMAs do not depend
+            // on the tile.
             constexpr uint32_t idesc = umma_idesc_bf16(kPairRows, BM);
             const uint16_t mask = static_cast<uint16_t>(3u << leader);
-            for (int i = (warp == kWarpMma ? 0 : 1); i < steps; i += 2) {
-                const int xs = i % kXStages, ab = i % kABufs, db = i % kDBufs;
-                if (!mbar_wait(&ready[xs], (i / kXStages) & 1)) break;
-                if (i >= kDBufs && !mbar_wait(&d_empty[db], ((i / kDBufs) - 1) & 1)) break;
+            RingPos<kXStages> xs;      // step g: ready[g % kXStages], its x stage, done[g % kXStages]
+            int ab = 0, db = 0;        // A buffer g % kABufs, accumulator g % kDBufs
+            uint32_t dph = 0u;         // bit b: parity of the next d_empty wait of accumulator b
+            bool have = false;         // step g's inputs were seen in the previous step
+            for (long long g = 0; g < total; ++g) {
+                if (!have) {
+                    if (!mbar_wait(&ready[xs.slot], xs.phase)) break;
+                    if (g >= kDBufs && !mbar_wait(&d_empty[db], (dph >> db) & 1u)) break;
+                }
+                if (g >= kDBufs) dph ^= 1u << db;
                 tc_fence_after();
-                const uint32_t b0 = smem_u32(smem + xs * kXBytes);
+                const uint32_t b0 = smem_u32(smem + xs.slot * kXBytes);
                 const uint32_t d = tmem_base + db * BM;
                 const uint32_t a = tmem_base + kACol0 + ab * kACols;
+                RingPos<kXStages> nx = xs;
+                nx.advance();
+                const int ndb = db ^ 1;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
+                for (int kk = 0; kk < 4; ++kk) {
                     const uint64_t bd = umma_desc_sw128(b0 + (kk >> 2) * kXAtom + (kk & 3) * 32);
                     umma_bf16_ts_pair(d, a + 8 * kk, bd, idesc, kk > 0);
                 }
-                umma_commit_pair(&done[xs], mask);
+                have = g + 1 < total && mbar_test_wait(&ready[nx.slot], nx.phase) &&
+                       (g + 1 < kDBufs || mbar_test_wait(&d_empty[ndb], (dph >> ndb) & 1u));
+#pragma unroll
+                for (int kk = 4; kk < 8; ++kk) {
+                    const uint64_t bd = umma_desc_sw128(b0 + (kk >> 2) * kXAtom + (kk & 3) * 32);
+                    umma_bf16_ts_pair(d, a + 8 * kk, bd, idesc, true);
+                }
+                umma_commit_pair(&done[xs.slot], mask);
+                xs = nx;
+                ab = (ab + 1) & (kABufs - 1);
+                db = ndb;
             }
         }
         __syncwarp();
@@ -303,57 +448,68 @@ __global__ void __launch_bounds__(kThreads, 1)
         regs_shrink<kRegsDeq>();
         // ------------------------------------------------------------ dequantisation (both CTAs)
         const int quarter = warp & 3, half = (warp - kWarpDeq) >> 2;
-        const long long row = row0 + quarter * 32 + lane;   // weight row n
-        const bool row_ok = row < p.N;
         const int rl = quarter * 32 + lane;                  // row within the CTA's codes tile
         const uint32_t sw = static_cast<uint32_t>((rl >> 1) & 3);   // 64-byte swizzle of that row
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + kACol0 + half * 32;
         pdl_wait();   // the bias-step coefficients come from the preparation kernel
-        const uint4 *bcrow = reinterpret_cast<const uint4 *>(p.bc + (row_ok ? row : 0) * static_cast<long long>(p.Kx));
-        for (int i = 0; i < steps; ++i) {
-            const int ab = i % kABufs;
-            uint32_t r[32];
-            if (i >= nbs) {
-                // chunks 2 half, 2 half + 1 (words 8 half .. 8 half + 7) of this row's codes
-                const int j = i - nbs, ws = j % kWStages;
-                if (!mbar_wait(&w_full[ws], (j / kWStages) & 1)) break;
-                const uint32_t wrow = smem_u32(smem + kOffW + ws * kWBytes) + rl * 64;
-                const uint4 c0 = lds128(wrow + (((2u * half) ^ sw) << 4));
-                const uint4 c1 = lds128(wrow + (((2u * half + 1u) ^ sw) << 4));
+        RingPos<kXStages> rs;   // step g: ready[g % kXStages]
+        RingPos<kXStages> fs;   // step g - kABufs: done[...], the MMAs that last read A buffer g % kABufs
+        RingPos<kWStages> cs;   // codes ring
+        int ab = 0;
+        long long g = 0;
+        bool ok = true;
+        long long t = tile0;
+        for (int k = 0; k < ntl && ok; ++k, t += tstride) {
+            const long long row = tile_coord(t, p.tiles_n, pair_rank).row0 + rl;   // weight row n
+            const bool row_ok = row < p.N;
+            const uint4 *bcrow = reinterpret_cast<const uint4 *>(p.bc + (row_ok ? row : 0) * static_cast<long long>(p.Kx));
+            for (int i = 0; i < steps; ++i, ++g) {
+                uint32_t r[32];
+                if (i >= nbs) {
+                    // chunks 2 half, 2 half + 1 (words 8 half .. 8 half + 7) of this row's codes
+                    if (!mbar_wait(&w_full[cs.slot], cs.phase)) { ok = false; break; }
+                    const uint32_t wrow = smem_u32(smem + kOffW + cs.slot * kWBytes) + rl * 64;
+                    const uint4 c0 = lds128(wrow + (((2u * half) ^ sw) << 4));
+                    const uint4 c1 = lds128(wrow + (((2u * half + 1u) ^ sw) << 4));
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&w_empty[cs.slot]);   // the codes are in registers
+                    cs.advance();
+                    if (g >= kABufs && !mbar_wait(&done[fs.slot], fs.phase)) { ok = false; break; }
+                    tc_fence_after();   // the tensor cores' reads of this buffer precede the stores below
+                    const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {   // word jj: k = 8 jj .. 8 jj + 7 -> columns 4 jj .. 4 jj + 3
+                        const uint32_t v = w[jj], v4 = v >> 4;
+                        r[4 * jj + 0] = bf16x2_plus128(v, v4, 0x0400u);
+                        r[4 * jj + 1] = bf16x2_plus128(v, v4, 0x0501u);
+                        r[4 * jj + 2] = bf16x2_plus128(v, v4, 0x0602u);
+                        r[4 * jj + 3] = bf16x2_plus128(v, v4, 0x0703u);
+                    }
+                } else {   // 64 coefficients of this column half (bias steps are few: loaded here)
+                    const int t = split + i * p.splits;
+                    uint4 v[8];
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj)
+                        v[jj] = row_ok ? ldg_nc_v4(bcrow + t * 16 + half * 8 + jj) : make_uint4(0, 0, 0, 0);
+                    if (g >= kABufs && !mbar_wait(&done[fs.slot], fs.phase)) { ok = false; break; }
+                    tc_fence_after();
+#pragma unroll
+                    for (int jj = 0; jj < 8; ++jj) {
+                        r[4 * jj + 0] = v[jj].x;
+                        r[4 * jj + 1] = v[jj].y;
+                        r[4 * jj + 2] = v[jj].z;
+                        r[4 * jj + 3] = v[jj].w;
+                    }
+                }
+                if (g >= kABufs) fs.advance();
+                tmem_st32(taddr + ab * kACols, r);
+                tmem_st_wait_regs(r);
+                tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(&w_empty[ws]);   // the codes are in registers
-                if (i >= kABufs && !mbar_wait(&done[(i - kABufs) % kXStages], ((i - kABufs) / kXStages) & 1)) break;
-                tc_fence_after();   // the tensor cores' reads of this buffer precede the stores below
-                const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {   // word jj: k = 8 jj .. 8 jj + 7 -> columns 4 jj .. 4 jj + 3
-                    const uint32_t v = w[jj], v4 = v >> 4;
-                    r[4 * jj + 0] = bf16x2_plus128(v, v4, 0x0400u);
-                    r[4 * jj + 1] = bf16x2_plus128(v, v4, 0x0501u);
-                    r[4 * jj + 2] = bf16x2_plus128(v, v4, 0x0602u);
-                    r[4 * jj + 3] = bf16x2_plus128(v, v4, 0x0703u);
-                }
-            } else {   // 64 coefficients of this column half (bias steps are few: loaded here)
-                const int t = split + i * p.splits;
-                uint4 v[8];
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj)
-                    v[jj] = row_ok ? ldg_nc_v4(bcrow + t * 16 + half * 8 + jj) : make_uint4(0, 0, 0, 0);
-                if (i >= kABufs && !mbar_wait(&done[(i - kABufs) % kXStages], ((i - kABufs) / kXStages) & 1)) break;
-                tc_fence_after();
-#pragma unroll
-                for (int jj = 0; jj < 8; ++jj) {
-                    r[4 * jj + 0] = v[jj].x;
-                    r[4 * jj + 1] = v[jj].y;
-                    r[4 * jj + 2] = v[jj].z;
-                    r[4 * jj + 3] = v[jj].w;
-                }
+                if (lane == 0) mbar_arrive_cluster(ready_l + 8 * rs.slot);
+                rs.advance();
+                ab = (ab + 1) & (kABufs - 1);
             }
-            tmem_st32(taddr + ab * kACols, r);
-            tmem_st_wait_regs(r);
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(ready_l + 8 * (i % kXStages));
         }
         named_bar_sync(kBarRegs, kThreads);
         regs_grow<kLaunchRegs>();
@@ -362,72 +518,81 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------ epilogue (both CTAs)
         const int quarter = warp & 3, half = (warp - kWarpEpi) >> 2;
         const int nl = quarter * 32 + lane;                         // weight row within the CTA
-        const long long row = row0 + nl;
-        const bool row_ok = row < p.N;
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * 64;
-        if (!p.static_weights) pdl_wait();   // scales are weights
-        {
-            // stage the scales of this CTA's rows ([128][G] BF16, contiguous in global memory)
-            // with coalesced loads; no load of this warp stays in flight across its arrivals
-            const int t = threadIdx.x - kWarpEpi * 32;
-            const long long rows = min(static_cast<long long>(BN), max(0ll, p.N - row0));
-            const long long elems = rows * G;
-            const uint16_t *src = p.scales + row0 * G;
-            const long long vec = (elems * 2) / 16;
-            for (long long v = t; v < vec; v += kEpiWarps * 32)
-                reinterpret_cast<uint4 *>(sc_smem)[v] = ldg_nc_v4(reinterpret_cast<const uint4 *>(src) + v);
-            for (long long e = vec * 8 + t; e < elems; e += kEpiWarps * 32) sc_smem[e] = __ldg(src + e);
-        }
-        named_bar_sync(kBarScales, kEpiWarps * 32);
-        const uint16_t *srow = sc_smem + nl * G;
-        float acc[64];
+        RingPos<kXStages> ds;   // step g: done[g % kXStages]
+        int db = 0;
+        bool ok = true;
+        // Every epilogue warp takes both named barriers of every tile, also after a failed
+        // wait, so that none is left waiting on a barrier that the others skipped.
+        long long t = tile0;
+        for (int k = 0; k < ntl; ++k, t += tstride) {
+            const TileCoord tc = tile_coord(t, p.tiles_n, pair_rank);
+            const int tile_m = tc.m;
+            const long long row0 = tc.row0;
+            const long long row = row0 + nl;
+            const bool row_ok = row < p.N;
+            const int sb = nsb == 2 ? (k & 1) : 0;
+            const uint32_t use = static_cast<uint32_t>(nsb == 2 ? (k >> 1) : k);
+            if (ok && !mbar_wait(&sc_full[sb], use & 1u)) ok = false;   // this tile's scales are staged
+            const uint16_t *srow = sc_smem + sb * BN * G + nl * G;
+            unsigned long long acc2[32];   // FP32 pairs: x rows 2j, 2j + 1 of this warp's 64
 #pragma unroll
-        for (int j = 0; j < 64; ++j) acc[j] = 0.f;
-        for (int i = 0; i < steps; ++i) {
-            const int db = i % kDBufs;
-            const float sc = (row_ok && i >= nbs) ? bf16_to_f32(srow[g0 + i - nbs]) : 1.f;
-            if (!mbar_wait(&done[i % kXStages], (i / kXStages) & 1)) break;
-            tc_fence_after();
-            uint32_t r0[32], r1[32];
-            tmem_ld32(taddr + db * BM, r0);
-            tmem_ld32(taddr + db * BM + 32, r1);
-            tmem_ld_wait_regs(r0);
-            tmem_ld_wait_regs(r1);   // both loads completed at the first wait; this only pins r1
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive_cluster(d_empty_l + 8 * db);
+            for (int j = 0; j < 32; ++j) acc2[j] = 0ull;
+            for (int i = 0; i < steps && ok; ++i) {
+                const float sc = (row_ok && i >= nbs) ? bf16_to_f32(srow[g0 + i - nbs]) : 1.f;
+                if (!mbar_wait(&done[ds.slot], ds.phase)) { ok = false; break; }
+                tc_fence_after();
+                uint32_t r[64];
+                tmem_ld64(taddr + db * BM, r);
+                tmem_ld_wait64(r);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive_cluster(d_empty_l + 8 * db);
+                const unsigned long long sc2 = f32x2(sc, sc);
+#pragma unroll
+                for (int j = 0; j < 32; ++j) ffma2(acc2[j], sc2, r[2 * j], r[2 * j + 1]);
+                ds.advance();
+                db ^= 1;
+            }
+            float acc[64];
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
-                acc[j] = fmaf(sc, __uint_as_float(r0[j]), acc[j]);
-                acc[32 + j] = fmaf(sc, __uint_as_float(r1[j]), acc[32 + j]);
+                acc[2 * j] = f32x2_lo(acc2[j]);
+                acc[2 * j + 1] = f32x2_hi(acc2[j]);
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sc_empty[sb]);   // this tile's scales are no longer read
+            if (k == 0) pdl_wait();   // y may still be read by the preceding kernel
+            const int m0 = tile_m * BM + half * 64;
+            if (p.splits > 1) {
+                // split-K (one tile per CTA): this CTA's partial, [x row][weight row] FP32,
+                // into the x stages, idle once the loop is over
+                float *part = reinterpret_cast<float *>(smem);
+#pragma unroll
+                for (int j = 0; j < 64; ++j) part[(half * 64 + j) * BN + nl] = acc[j];
+            } else if (p.tma_store) {
+                // the tile, [x row][weight row] BF16, into the staging buffer, then one TMA store
+                // that overlaps the next tile's main loop
+                if (warp == kWarpEpi && lane == 0) bulk_wait_read_all();   // the previous store read it
+                named_bar_sync(kBarEpi, kEpiWarps * 32);
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    out_tile[(half * 64 + j) * BN + nl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+                fence_proxy_async_smem();   // the async proxy reads the tile
+                named_bar_sync(kBarEpi, kEpiWarps * 32);
+                if (ok && warp == kWarpEpi && lane == 0) {
+                    tma_store_2d(&tm_y, out_tile, static_cast<int>(row0), tile_m * BM);
+                    bulk_commit_group();
+                }
+            } else if (row_ok && ok) {
+#pragma unroll
+                for (int j = 0; j < 64; ++j)
+                    if (m0 + j < p.M)
+                        p.y[static_cast<long long>(m0 + j) * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
             }
         }
-        pdl_wait();   // y may still be read by the preceding kernel
-        const int m0 = tile_m * BM + half * 64;
-        if (p.splits > 1) {
-            // split-K: this CTA's partial, [x row][weight row] FP32, into the (idle) x stages
-            float *part = reinterpret_cast<float *>(smem);
-#pragma unroll
-            for (int j = 0; j < 64; ++j) part[(half * 64 + j) * BN + nl] = acc[j];
-        } else if (p.tma_store) {
-            // the tile, [x row][weight row] BF16, into the (idle) x stages, then one TMA store
-            uint16_t *tile = reinterpret_cast<uint16_t *>(smem);
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-                tile[(half * 64 + j) * BN + nl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
-            fence_proxy_async_smem();   // the async proxy reads the tile
-            named_bar_sync(kBarScales, kEpiWarps * 32);
-            if (warp == kWarpEpi && lane == 0) {
-                tma_store_2d(&tm_y, tile, static_cast<int>(row0), tile_m * BM);
-                bulk_commit_group();
-                bulk_wait_all();   // shared memory is released, and y written, before the CTA ends
-            }
-        } else if (row_ok) {
-#pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (m0 + j < p.M)
-                    p.y[static_cast<long long>(m0 + j) * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
-        }
+        if (p.tma_store && warp == kWarpEpi && lane == 0)
+            bulk_wait_all();   // y written, and shared memory released, before the CTA ends
         regs_shrink<kLaunchRegs>();            // released first ...
         named_bar_arrive(kBarRegs, kThreads);  // ... then the other warpgroups grow back into it
     }
@@ -442,10 +607,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     // Every CTA of the cluster is done with its peers' barriers and shared memory only
     // after this barrier: none leaves while another may still signal or read it.
     cluster_sync_all();
-    if (p.splits > 1) {
+    if (p.splits > 1 && ntl == 1) {
         // Split-K reduction over the S pairs of the cluster: the CTAs with this pair rank
         // hold the S partials of the same 128 weight rows; the one of split r sums x rows
         // [r*R, (r+1)*R) of them, in split order, through distributed shared memory.
+        const TileCoord tc = tile_coord(tile0, p.tiles_n, pair_rank);
+        const int tile_m = tc.m;
+        const long long row0 = tc.row0;
         if (warp >= kWarpEpi) {
             const int S = p.splits;
             const int rows_per = (BM + S - 1) / S;

@@ -43,6 +43,7 @@ struct DeviceInfo {
     int status = W4A16_OK;
     int sms = 0;
     bool gemm_ok = false;     // the GEMM's register split fits its launch allocation
+    int gemm_clusters = 0;    // CTA pairs of the GEMM resident at once (its persistent grid)
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
 };
 
@@ -93,6 +94,23 @@ int device_setup(int dev, DeviceInfo **out) {
                 e = cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          gm::smem_bytes(gm::kMaxGroups));
             if (e != cudaSuccess) return cuda_fail(e);
+            // how many CTA pairs of the GEMM the device holds at once: the persistent grid
+            // never exceeds it, so that no pair waits for another to finish
+            cudaLaunchConfig_t occ = {};
+            occ.gridDim = dim3(2, 1, 1);
+            occ.blockDim = dim3(gm::kThreads, 1, 1);
+            occ.dynamicSmemBytes = gm::smem_bytes(gm::kMaxGroups);
+            cudaLaunchAttribute cl;
+            cl.id = cudaLaunchAttributeClusterDimension;
+            cl.val.clusterDim.x = 2;
+            cl.val.clusterDim.y = 1;
+            cl.val.clusterDim.z = 1;
+            occ.attrs = &cl;
+            occ.numAttrs = 1;
+            int clusters = 0;
+            e = cudaOccupancyMaxActiveClusters(&clusters, gm::gemm_kernel, &occ);
+            if (e != cudaSuccess) return cuda_fail(e);
+            d.gemm_clusters = clusters > 0 ? clusters : d.sms / 2;
         }
         d.ready = true;
     }
@@ -307,8 +325,14 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
     pl->path = W4A16_PATH_GEMM;
     pl->splits = static_cast<int32_t>(splits);
     pl->grid_x = static_cast<int32_t>(2 * splits);   // pairs of the splits of a tile: one cluster
-    pl->grid_y = static_cast<int32_t>(tn);
-    pl->grid_z = static_cast<int32_t>(tm);
+    if (splits == 1) {
+        // persistent: one CTA pair per two SMs, each looping over tiles
+        pl->grid_y = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(tm * tn, sms / 2)));
+        pl->grid_z = 1;
+    } else {
+        pl->grid_y = static_cast<int32_t>(tn);
+        pl->grid_z = static_cast<int32_t>(tm);
+    }
     pl->block = gm::kThreads;
     pl->smem_bytes = gm::smem_bytes(static_cast<int>(G));
     pl->cluster = static_cast<int32_t>(2 * splits);
@@ -454,10 +478,14 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     kp.G = G;
     kp.Kx = Kx;
     kp.splits = pl.splits;
+    kp.tiles = pl.tiles;
+    kp.tiles_n = static_cast<int>((p.N + gm::kPairRows - 1) / gm::kPairRows);
     kp.static_weights = static_weights ? 1 : 0;
     kp.tma_store = tma_store ? 1 : 0;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(pl.grid_x, pl.grid_y, pl.grid_z);
+    // a persistent grid is capped at the pairs the device holds at once
+    const int grid_y = pl.splits == 1 ? std::max(1, std::min(pl.grid_y, d->gemm_clusters)) : pl.grid_y;
+    cfg.gridDim = dim3(pl.grid_x, grid_y, pl.grid_z);
     cfg.blockDim = dim3(pl.block, 1, 1);
     cfg.dynamicSmemBytes = pl.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);

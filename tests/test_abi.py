@@ -133,13 +133,17 @@ def test_streamk_owner_matches_brute_force():
                                                  (509, 4096, 9728, 1), (129, 1000, 9728, 4)])
 def test_gemm_split_plan(M, N, K, expect_splits):
     """Tiles of 256 weight rows x 128 x rows, each on a CTA pair; K is split only while
-    the pairs leave SMs idle, and a tile's splits form one cluster of 2 x splits CTAs."""
+    the pairs leave SMs idle, and a tile's splits form one cluster of 2 x splits CTAs.
+    Without a split the grid is persistent: one pair per two SMs, looping over the tiles."""
     pl = w4.w4a16_plan(M, N, K, sm_count=148)
     assert pl["path"] == w4.PATH_GEMM
     assert pl["splits"] == expect_splits and pl["cluster"] == 2 * expect_splits
     tiles = -(-M // 128) * -(-N // 256)
     assert pl["tiles"] == tiles
-    assert pl["grid_x"] * pl["grid_y"] * pl["grid_z"] == 2 * tiles * expect_splits
+    if expect_splits == 1:
+        assert (pl["grid_x"], pl["grid_y"], pl["grid_z"]) == (2, min(tiles, 74), 1)
+    else:
+        assert pl["grid_x"] * pl["grid_y"] * pl["grid_z"] == 2 * tiles * expect_splits
     assert pl["splits"] <= 4 and pl["splits"] <= K // 128
     assert pl["cluster"] <= 8
 
