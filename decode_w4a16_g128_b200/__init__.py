@@ -31,6 +31,7 @@ ERR_TIMEOUT = 7
 PATH_AUTO = 0
 PATH_MATVEC = 1
 PATH_GEMM = 2
+PATH_MATVEC_ROWS = 3
 
 FLAG_NO_PDL = 1
 FLAG_STATIC_WEIGHTS = 2

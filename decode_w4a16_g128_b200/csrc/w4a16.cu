@@ -19,6 +19,7 @@
 
 #include "gemm.cuh"
 #include "matvec.cuh"
+#include "rows.cuh"
 
 namespace w4a16 {
 namespace {
@@ -86,6 +87,8 @@ int device_setup(int dev, DeviceInfo **out) {
             if (e != cudaSuccess) return cuda_fail(e);
             d.gemm_ok = fa.numRegs * gm::kThreads >=
                         128 * (gm::kRegsCtl + 2 * gm::kRegsDeq + 2 * gm::kRegsEpi);
+            e = cudaFuncSetAttribute(mvr::rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mvr::kBudget);
+            if (e != cudaSuccess) return cuda_fail(e);
             e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      int(kMatvecBudget));
             if (e == cudaSuccess)   // one carveout for every launch: no reconfiguration between them
@@ -232,6 +235,9 @@ int choose_path(int64_t M, const w4a16_options *opt, int *path) {
         *path = W4A16_PATH_MATVEC;
     } else if (req == W4A16_PATH_GEMM) {
         *path = W4A16_PATH_GEMM;
+    } else if (req == W4A16_PATH_MATVEC_ROWS) {
+        if (M > mvr::kMaxM) return W4A16_ERR_UNSUPPORTED;
+        *path = W4A16_PATH_MATVEC_ROWS;
     } else {
         return W4A16_ERR_INVALID_ARG;
     }
@@ -341,10 +347,35 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
     pl->workspace_bytes = (M + N) * gm::xs_cols(static_cast<int>(G)) * 2;   // bias-step operands
 }
 
+// Row-block matvec: ceil(N / (8 noct)) CTAs of 8 noct whole weight rows each.
+void plan_rows(int64_t N, int64_t K, int noct, w4a16_plan_info *pl) {
+    const int64_t oct = (N + 7) / 8;
+    std::memset(pl, 0, sizeof(*pl));
+    pl->path = W4A16_PATH_MATVEC_ROWS;
+    pl->splits = 1;
+    pl->grid_x = static_cast<int32_t>((oct + noct - 1) / noct);
+    pl->grid_y = pl->grid_z = 1;
+    pl->block = mvr::kThreads;
+    pl->smem_bytes = static_cast<int32_t>(mvr::smem_bytes(noct, static_cast<int>(K / 128)));
+    pl->cluster = 1;
+    pl->tiles = pl->grid_x;   // row blocks
+    pl->units = oct;          // weight-row octets
+    pl->workspace_bytes = 0;
+}
+
 int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a16_plan_info *pl) {
     int path = 0;
     int rc = choose_path(M, opt, &path);
     if (rc) return rc;
+    const int req = opt ? opt->path : W4A16_PATH_AUTO;
+    const int noct = mvr::plan_octets(N, K, sms);
+    if (path == W4A16_PATH_MATVEC_ROWS && noct == 0) return W4A16_ERR_UNSUPPORTED;
+    if (path == W4A16_PATH_MATVEC && req == W4A16_PATH_AUTO && !(opt && opt->workers > 0) && noct > 0)
+        path = W4A16_PATH_MATVEC_ROWS;
+    if (path == W4A16_PATH_MATVEC_ROWS) {
+        plan_rows(N, K, noct, pl);
+        return W4A16_OK;
+    }
     if (path == W4A16_PATH_MATVEC) {
         plan_matvec(M, N, K, sms, opt, pl);
         return W4A16_OK;
@@ -373,6 +404,40 @@ int encode_2d(DeviceInfo *d, CUtensorMap *map, CUtensorMapDataType type, const v
         return W4A16_ERR_CUDA;
     }
     return W4A16_OK;
+}
+
+int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void *stream, bool pdl,
+                bool static_weights) {
+    const int G = static_cast<int>(p.K / 128);
+    const int noct = static_cast<int>((pl.units + pl.grid_x - 1) / pl.grid_x);
+    CUtensorMap tm_w;
+    // codes: [N, K/8] uint32, boxes of 32 words (128 B: two groups) x 8 noct rows, 128-byte swizzle
+    int rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 32,
+                       static_cast<uint32_t>(8 * noct), CU_TENSOR_MAP_SWIZZLE_128B);
+    if (rc) return rc;
+    mvr::Params kp;
+    kp.x = static_cast<const uint16_t *>(p.x);
+    kp.scales = static_cast<const uint16_t *>(p.scales);
+    kp.biases = static_cast<const uint16_t *>(p.biases);
+    kp.y = static_cast<uint16_t *>(p.y);
+    kp.M = static_cast<int>(p.M);
+    kp.N = static_cast<int>(p.N);
+    kp.K = static_cast<int>(p.K);
+    kp.G = G;
+    kp.noct = noct;
+    kp.static_weights = static_weights ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(pl.grid_x, 1, 1);
+    cfg.blockDim = dim3(pl.block, 1, 1);
+    cfg.dynamicSmemBytes = pl.smem_bytes;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, mvr::rows_kernel, tm_w, kp);
+    return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
 int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan_info &pl, void *stream,
@@ -527,6 +592,7 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     if (rc) return rc;
     const bool pdl = !(opt && (opt->flags & W4A16_FLAG_NO_PDL));
     const bool static_weights = opt && (opt->flags & W4A16_FLAG_STATIC_WEIGHTS);
+    if (pl.path == W4A16_PATH_MATVEC_ROWS) return launch_rows(d, p, pl, stream, pdl, pdl && static_weights);
     if (pl.path == W4A16_PATH_MATVEC) {
         Workspace *ws = nullptr;
         rc = workspace_get(dev, stream, size_t(pl.grid_x) * mv::kPartialFloats, pl.tiles, &ws);

@@ -64,7 +64,12 @@ enum w4a16_status_code {
 enum w4a16_path {
     W4A16_PATH_AUTO = 0,        /* M <= 8: matvec; M > 8: tensor-core GEMM (Task 1 dispatch rule) */
     W4A16_PATH_MATVEC = 1,      /* weight-streaming matvec, M <= 8 only                           */
-    W4A16_PATH_GEMM = 2         /* tcgen05 tensor-core GEMM, any M >= 1                            */
+    W4A16_PATH_GEMM = 2,        /* tcgen05 tensor-core GEMM, any M >= 1                            */
+    W4A16_PATH_MATVEC_ROWS = 3  /* row-block matvec, M <= 8: each CTA owns whole weight rows over all
+                                   of K (no cross-CTA sum), at most two CTAs per SM; only where such
+                                   a split fits (else W4A16_ERR_UNSUPPORTED).  W4A16_PATH_AUTO takes
+                                   it for M <= 8 when it fits and no worker count is given, the
+                                   stream-K matvec (W4A16_PATH_MATVEC) otherwise                   */
 };
 
 /*

@@ -97,15 +97,61 @@ def test_bad_options():
 
 
 def test_dispatch_rule():
-    """M <= 8 streams weights through the matvec; larger M goes to the tensor-core GEMM."""
+    """M <= 8 streams weights through a matvec (the row-block one where a CTA's whole rows
+    fit, the stream-K one otherwise); larger M goes to the tensor-core GEMM."""
     for M in range(1, 9):
-        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148)["path"] == w4.PATH_MATVEC
+        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148)["path"] == w4.PATH_MATVEC_ROWS
+        assert w4.w4a16_plan(M, 151936, 2560, sm_count=148)["path"] == w4.PATH_MATVEC
+        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148, workers=64)["path"] == w4.PATH_MATVEC
+    assert w4.w4a16_plan(9, 4096, 2560, sm_count=148)["path"] == w4.PATH_GEMM
+
+
+@pytest.mark.parametrize("N,K,noct,grid", [(1024, 2560, 1, 128), (4096, 2560, 4, 128), (2560, 4096, 3, 107),
+                                           (9728, 2560, 9, 136), (2560, 9728, 2, 160), (1000, 256, 1, 125),
+                                           (8, 128, 1, 1), (1, 128, 1, 1)])
+def test_rows_plan(N, K, noct, grid):
+    """Row-block matvec: CTAs of 8 noct whole weight rows, as few as one pass needs, at most
+    two per SM, each within 110 KB of shared memory so that two fit on an SM."""
+    pl = w4.w4a16_plan(1, N, K, sm_count=148)
+    assert pl["path"] == w4.PATH_MATVEC_ROWS
+    assert pl["block"] == 288            # producer warp + 8 compute warps
+    assert pl["units"] == -(-N // 8)     # weight-row octets
+    assert pl["grid_x"] == grid == -(-pl["units"] // noct)
+    assert pl["grid_x"] <= 2 * 148
+    assert pl["smem_bytes"] <= 110 * 1024 and 2 * (pl["smem_bytes"] + 1024) <= 228 * 1024
+    assert pl["workspace_bytes"] == 0
+
+
+def test_rows_plan_limits():
+    # the vocabulary projection does not fit two CTAs per SM: stream-K there
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_plan(1, 151936, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148)
+    assert e.value.status == w4.ERR_UNSUPPORTED
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_plan(9, 4096, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148)
+    assert e.value.status == w4.ERR_UNSUPPORTED
+    # the chosen split: as few CTAs as possible; one octet more per CTA would exceed 110 KB
+    def smem(noct, G):   # codes boxes (or the warps' partial sums), scales, biases, barriers, slack
+        boxes = (G + 1) // 2
+        work = max(8 * noct * 128 * boxes, 4 * 8 * 8 * noct * 8)
+        return work + 2 * ((16 * noct * G + 15) // 16 * 16) + 8 * (boxes + 1) + 1024
+    for N in (8, 100, 1000, 2560, 4096, 9728, 20000):
+        for K in (128, 256, 2560, 4096, 9728, 16384):
+            try:
+                pl = w4.w4a16_plan(1, N, K, path=w4.PATH_MATVEC_ROWS, sm_count=148)
+            except w4.W4A16Error:
+                continue
+            oct_, G = -(-N // 8), K // 128
+            noct = -(-oct_ // pl["grid_x"])
+            assert pl["grid_x"] <= 296 and noct <= 9 and pl["smem_bytes"] == smem(noct, G)
+            if noct < min(-(-oct_ // 148), 9):
+                assert smem(noct + 1, G) > 110 * 1024, (N, K, noct)
 
 
 @pytest.mark.parametrize("N,K", [(1024, 2560), (4096, 2560), (2560, 4096), (9728, 2560), (2560, 9728),
                                  (151936, 2560), (1000, 256), (8, 128)])
 def test_matvec_plan(N, K):
-    pl = w4.w4a16_plan(1, N, K, sm_count=148)
+    pl = w4.w4a16_plan(1, N, K, path=w4.PATH_MATVEC, sm_count=148)
     assert pl["block"] == 672   # producer warp, 4 x-preparation warps, 16 consumer warps
     assert pl["tiles"] == -(-N // 256)   # 16 consumer warps x 16 rows
     assert pl["units"] == pl["tiles"] * (K // 128)
@@ -171,6 +217,6 @@ def test_gemm_k_limit():
 def test_matvec_default_workers(N, K, expect):
     """Persistent CTAs of the matvec: fewer than the SMs for small and mid-size weights (the
     next call's CTAs start on the free SMs), every SM for the vocabulary projection."""
-    pl = w4.w4a16_plan(1, N, K, sm_count=148)
+    pl = w4.w4a16_plan(1, N, K, path=w4.PATH_MATVEC, sm_count=148)
     assert pl["path"] == w4.PATH_MATVEC and pl["grid_x"] == expect
     assert w4.w4a16_plan(1, N, K, sm_count=148, workers=17)["grid_x"] == min(17, pl["units"])

@@ -4,7 +4,9 @@ Covers the decode configuration (M in {1, 2, 4, 8} over the seven Qwen3-4B
 projection shapes) element by element, ragged row counts, every M up to 8,
 exact integer problems (bit-exact on every worker split), determinism, the
 stream-K split at many worker counts, guard bands around y, and a stream
-other than the default one.
+other than the default one.  These tests force the stream-K kernel
+(W4A16_PATH_MATVEC) where the automatic choice would take the row-block one;
+test_rows_gpu.py covers that kernel.
 """
 import numpy as np
 import pytest
@@ -37,7 +39,7 @@ def run(prob, **kw):
 @pytest.mark.parametrize("name,K,N", synth.QWEN3_4B_PROJECTIONS, ids=[p[0] for p in synth.QWEN3_4B_PROJECTIONS])
 def test_decode_projection(M, name, K, N):
     prob = synth.make_problem(M, N, K)
-    got = run(prob)
+    got = run(prob, path=w4.PATH_MATVEC)
     r = assert_close(got, oracle_y(prob), f"{name} M={M}")
     assert r["exact"] > 0.9 * r["n"]
 
@@ -46,7 +48,7 @@ def test_decode_projection(M, name, K, N):
 @pytest.mark.parametrize("N,K", [(8, 128), (129, 256), (1000, 2560), (1001, 384), (130, 9728), (4097, 128)])
 def test_ragged_shapes(M, N, K):
     prob = synth.make_problem(M, N, K, outliers=True)
-    assert_close(run(prob), oracle_y(prob), f"M={M} N={N} K={K}")
+    assert_close(run(prob, path=w4.PATH_MATVEC), oracle_y(prob), f"M={M} N={N} K={K}")
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 24, 384), (5, 130, 640), (8, 257, 1024), (3, 1, 256), (8, 1000, 512)])
