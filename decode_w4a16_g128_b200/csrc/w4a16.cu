@@ -88,6 +88,10 @@ int device_setup(int dev, DeviceInfo **out) {
             d.gemm_ok = fa.numRegs * gm::kThreads >=
                         128 * (gm::kRegsCtl + 2 * gm::kRegsDeq + 2 * gm::kRegsEpi);
             e = cudaFuncSetAttribute(mvr::rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mvr::kBudget);
+            // the largest shared-memory carveout: two CTAs per SM (without it the driver
+            // picks a split that holds one), and the same split as the other kernels
+            if (e == cudaSuccess)
+                e = cudaFuncSetAttribute(mvr::rows_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
             if (e != cudaSuccess) return cuda_fail(e);
             e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      int(kMatvecBudget));
