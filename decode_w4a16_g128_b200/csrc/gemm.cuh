@@ -141,58 +141,67 @@ struct Params {
 
 // ------------------------------------------------------------------ preparation: bias-step operands
 
-// Items [0, M G): Xs[m, 6g + j] = Xs[m, 6g + 3 + j] = piece j of X[m,g] =
-// sum_{k in g} x[m,k] (FP32, k ascending), X = p0 + p1 + p2 exactly with
+// Xs[m, 6g + j] = Xs[m, 6g + 3 + j] = piece j of X[m,g] = sum_{k in g} x[m,k]
+// (FP32: each lane of a half-warp sums 8 consecutive values, then the 16 lanes
+// in a fixed tree), X = p0 + p1 + p2 exactly with
 // p0 = bf16(X), p1 = bf16(X - p0), p2 = X - p0 - p1 (exact in BF16).
-// Items [M G, M G + N G): Bc[n, 6g + j] = b[n,g], Bc[n, 6g + 3 + j] = -128 s[n,g].
+// Bc[n, 6g + j] = b[n,g], Bc[n, 6g + 3 + j] = -128 s[n,g] (one thread per (n, g)).
 // The last group of a row also writes the zero padding 6G .. Kx-1.
 __global__ void __launch_bounds__(256) prep_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
                                                    const uint16_t *__restrict__ biases, uint16_t *__restrict__ xs,
                                                    uint16_t *__restrict__ bc, int M, int N, int G, int Kx) {
     pdl_launch_dependents();   // the GEMM may start its prologue
     pdl_wait();                // x may come from the previous kernel of the stream
-    const long long mg = static_cast<long long>(M) * G;
-    const long long total = mg + static_cast<long long>(N) * G;
     const long long K = static_cast<long long>(G) * 128;
-    for (long long idx = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; idx < total;
-         idx += static_cast<long long>(gridDim.x) * blockDim.x) {
-        const bool is_x = idx < mg;
-        const long long item = is_x ? idx : idx - mg;
-        const long long r = item / G;
-        const int g = static_cast<int>(item - r * G);
-        uint32_t w0, w1, w2;
-        if (is_x) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(x + r * K + g * 128);
-            float sum = 0.f;
-#pragma unroll 4
-            for (int i = 0; i < 16; ++i) {
-                const uint4 v = __ldg(src + i);
-                const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    const long long threads = static_cast<long long>(gridDim.x) * blockDim.x;
+    const long long tid = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x;
+    const int lane = threadIdx.x & 31, half = lane >> 4, l16 = lane & 15;
+    // x: each half-warp sums one (row m, group g): one 16-byte load per lane, then the
+    // 16 lanes' sums; the loop bound is warp-uniform so that every lane takes each shuffle
+    const long long mg = static_cast<long long>(M) * G;
+    for (long long wu = (tid >> 5) * 2; wu < mg; wu += (threads >> 5) * 2) {
+        const long long u = wu + half;
+        const bool live = u < mg;
+        const long long r = live ? u / G : 0;
+        const int g = live ? static_cast<int>(u - r * G) : 0;
+        float sum = 0.f;
+        if (live) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4 *>(x + r * K + g * 128) + l16);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    sum += bf16_lo_to_f32(w[j]);
-                    sum += bf16_hi_to_f32(w[j]);
-                }
+            for (int j = 0; j < 4; ++j) {
+                sum += bf16_lo_to_f32(w[j]);
+                sum += bf16_hi_to_f32(w[j]);
             }
+        }
+#pragma unroll
+        for (int o = 1; o < 16; o <<= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+        if (live && l16 == 0) {
             const uint32_t p0 = __bfloat16_as_ushort(__float2bfloat16_rn(sum));
             const float r1 = sum - bf16_to_f32(p0);
             const uint32_t p1 = __bfloat16_as_ushort(__float2bfloat16_rn(r1));
             const uint32_t p2 = __bfloat16_as_ushort(__float2bfloat16_rn(r1 - bf16_to_f32(p1)));
-            w0 = p0 | (p1 << 16);
-            w1 = p2 | (p0 << 16);
-            w2 = p1 | (p2 << 16);
-        } else {
-            const uint32_t b = __ldg(biases + r * G + g);
-            const uint32_t t = __bfloat16_as_ushort(__float2bfloat16_rn(-128.f * bf16_to_f32(__ldg(scales + r * G + g))));
-            w0 = b | (b << 16);
-            w1 = b | (t << 16);
-            w2 = t | (t << 16);
+            uint16_t *row = xs + r * Kx;
+            uint32_t *dst = reinterpret_cast<uint32_t *>(row + kBiasCoef * g);   // 4-byte aligned
+            dst[0] = p0 | (p1 << 16);
+            dst[1] = p2 | (p0 << 16);
+            dst[2] = p1 | (p2 << 16);
+            if (g == G - 1)
+                for (int c = kBiasCoef * G; c < Kx; c += 2) *reinterpret_cast<uint32_t *>(row + c) = 0u;
         }
-        uint16_t *row = (is_x ? xs : bc) + r * Kx;
-        uint32_t *dst = reinterpret_cast<uint32_t *>(row + kBiasCoef * g);   // 4-byte aligned
-        dst[0] = w0;
-        dst[1] = w1;
-        dst[2] = w2;
+    }
+    // coefficients: one thread per (weight row n, group g)
+    const long long ng = static_cast<long long>(N) * G;
+    for (long long item = tid; item < ng; item += threads) {
+        const long long r = item / G;
+        const int g = static_cast<int>(item - r * G);
+        const uint32_t b = __ldg(biases + r * G + g);
+        const uint32_t t = __bfloat16_as_ushort(__float2bfloat16_rn(-128.f * bf16_to_f32(__ldg(scales + r * G + g))));
+        uint16_t *row = bc + r * Kx;
+        uint32_t *dst = reinterpret_cast<uint32_t *>(row + kBiasCoef * g);
+        dst[0] = b | (b << 16);
+        dst[1] = b | (t << 16);
+        dst[2] = t | (t << 16);
         if (g == G - 1)
             for (int c = kBiasCoef * G; c < Kx; c += 2) *reinterpret_cast<uint32_t *>(row + c) = 0u;
     }

@@ -521,7 +521,8 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     // 1. bias-step operands: group sums of x and the matching weight coefficients
     uint16_t *bc = ws->xs + size_t(p.M) * Kx;
     {
-        const long long items = (p.M + p.N) * G;
+        // threads: 16 per (x row, group), one per (weight row, group); the kernel loops
+        const long long items = std::max<long long>(p.M * G * 16, p.N * G);
         const long long blocks = std::min<long long>((items + 255) / 256, static_cast<long long>(d->sms) * 8);
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(static_cast<unsigned>(std::max<long long>(blocks, 1)), 1, 1);
