@@ -354,10 +354,12 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
 // Row-block matvec: ceil(N / (8 noct)) CTAs of 8 noct whole weight rows each.
 void plan_rows(int64_t N, int64_t K, int noct, w4a16_plan_info *pl) {
     const int64_t oct = (N + 7) / 8;
+    const int64_t grid = (oct + noct - 1) / noct;
+    noct = static_cast<int>((oct + grid - 1) / grid);   // the same CTA count may need fewer octets each
     std::memset(pl, 0, sizeof(*pl));
     pl->path = W4A16_PATH_MATVEC_ROWS;
     pl->splits = 1;
-    pl->grid_x = static_cast<int32_t>((oct + noct - 1) / noct);
+    pl->grid_x = static_cast<int32_t>(grid);
     pl->grid_y = pl->grid_z = 1;
     pl->block = mvr::kThreads;
     pl->smem_bytes = static_cast<int32_t>(mvr::smem_bytes(noct, static_cast<int>(K / 128)));

@@ -135,6 +135,11 @@ def test_rows_plan_limits():
         boxes = (G + 1) // 2
         work = max(8 * noct * 128 * boxes, 4 * 8 * 8 * noct * 8)
         return work + 2 * ((16 * noct * G + 15) // 16 * 16) + 8 * (boxes + 1) + 1024
+    # 9 octets on 2 SMs, K = 5376: 5 octets per CTA exceed 110 KB, 4 fit, and the 3 CTAs
+    # that 4 octets need hold 3 octets each: the plan describes what is launched
+    pl = w4.w4a16_plan(1, 72, 5376, path=w4.PATH_MATVEC_ROWS, sm_count=2)
+    assert smem(5, 42) > 110 * 1024 >= smem(4, 42)
+    assert pl["grid_x"] == 3 and pl["smem_bytes"] == smem(3, 42)
     for N in (8, 100, 1000, 2560, 4096, 9728, 20000):
         for K in (128, 256, 2560, 4096, 9728, 16384):
             try:
