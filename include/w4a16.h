@@ -132,12 +132,14 @@ int w4a16_matmul_ex(const void *x, const uint32_t *wq, const void *scales,
 typedef struct w4a16_plan_info {
     int32_t path;            /* enum w4a16_path chosen                                  */
     int32_t splits;          /* GEMM K splits (a cluster holds 2 x splits CTAs); 1 for the matvec */
-    int32_t grid_x, grid_y, grid_z;
+    int32_t grid_x, grid_y, grid_z;   /* GEMM without a K split: a persistent grid of at most
+                                         one CTA pair per two SMs, each pair looping over tiles */
     int32_t block;           /* threads per CTA                                         */
     int32_t smem_bytes;      /* dynamic shared memory per CTA                           */
     int32_t cluster;         /* CTAs per cluster (1 = no cluster)                       */
-    int64_t tiles;           /* output tiles                                            */
-    int64_t units;           /* matvec: (row tile x 128-group) work units               */
+    int64_t tiles;           /* output tiles (row-block matvec: row blocks, one per CTA) */
+    int64_t units;           /* stream-K matvec: (row tile x 128-group) work units;
+                                row-block matvec: weight-row octets                     */
     int64_t workspace_bytes; /* library workspace the call needs                        */
 } w4a16_plan_info;
 
