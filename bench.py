@@ -611,9 +611,9 @@ def detail(args, entries, calls, stream, pk):
         rows.append({"M": M, "proj": name, "N": N, "K": K, "us": round(us, 3), "GB/s": round(gb, 1),
                      "frac_hbm": round(gb / pk["hbm_gbs"], 3)})
         del g, copies
-    out = os.path.join(ROOT, "gpurun_out") if os.path.isdir(os.path.join(ROOT, "gpurun_out")) else ROOT
-    with open(os.path.join(out, "bench_detail.json"), "w") as f:
-        json.dump(rows, f, indent=1)
+    if args.detail:
+        with open(args.detail, "w") as f:
+            json.dump(rows, f, indent=1)
     for r in rows:
         print(json.dumps(r), file=sys.stderr)
 
@@ -625,7 +625,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=("ours", "reference"), default="ours")
     ap.add_argument("--mode", choices=("bench", "profile"), default="bench")
-    ap.add_argument("--detail", action="store_true", help="also time every call on its own")
+    ap.add_argument("--detail", default="", metavar="PATH",
+                    help="also time every decode call on its own and write the table to PATH (JSON)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the M > 8 measurements")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="time bound of the CPU baseline sample")

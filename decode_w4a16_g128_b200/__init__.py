@@ -45,14 +45,16 @@ class W4A16Error(RuntimeError):
 
 class Options(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("splits", ctypes.c_int32), ("workers", ctypes.c_int32),
-                ("sm_count", ctypes.c_int32), ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
+                ("sm_count", ctypes.c_int32), ("flags", ctypes.c_int32), ("row_blocks", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 2)]
 
 
 class PlanInfo(ctypes.Structure):
     _fields_ = [("path", ctypes.c_int32), ("splits", ctypes.c_int32), ("grid_x", ctypes.c_int32),
                 ("grid_y", ctypes.c_int32), ("grid_z", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("cluster", ctypes.c_int32), ("tiles", ctypes.c_int64),
-                ("units", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64)]
+                ("units", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64), ("row_blocks", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:
@@ -137,20 +139,20 @@ def w4a16_matmul(x, wq, scales, biases, y=None, stream=None):
     return y
 
 
-def make_options(path=PATH_AUTO, splits=0, workers=0, sm_count=0, flags=0) -> Options:
-    return Options(int(path), int(splits), int(workers), int(sm_count), int(flags))
+def make_options(path=PATH_AUTO, splits=0, workers=0, sm_count=0, flags=0, row_blocks=0) -> Options:
+    return Options(int(path), int(splits), int(workers), int(sm_count), int(flags), int(row_blocks))
 
 
 def w4a16_matmul_ex(x, wq, scales, biases, y=None, stream=None, path=PATH_AUTO, splits=0, workers=0,
-                    flags=0):
-    """w4a16_matmul with a forced path / split count / worker count."""
+                    flags=0, row_blocks=0):
+    """w4a16_matmul with a forced path / split count / worker count / row blocks per CTA."""
     import torch
     M, N, K = _check_tensors(x, wq, scales, biases, y)
     if y is None:
         y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
     elif tuple(y.shape) != (M, N):
         raise ValueError("y must be [M, N]")
-    opt = make_options(path, splits, workers, 0, flags)
+    opt = make_options(path, splits, workers, 0, flags, row_blocks)
     _check(lib.w4a16_matmul_ex(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(y), M, N, K,
                                _stream_handle(stream), ctypes.byref(opt)), "w4a16_matmul_ex")
     return y
@@ -186,11 +188,11 @@ def w4a16_matvec_noalloc(x, wq, scales, biases, y, stream=None):
     return y
 
 
-def w4a16_plan(M: int, N: int, K: int, path=PATH_AUTO, splits=0, workers=0, sm_count=0) -> dict:
-    opt = make_options(path, splits, workers, sm_count)
+def w4a16_plan(M: int, N: int, K: int, path=PATH_AUTO, splits=0, workers=0, sm_count=0, row_blocks=0) -> dict:
+    opt = make_options(path, splits, workers, sm_count, 0, row_blocks)
     info = PlanInfo()
     _check(lib.w4a16_plan(M, N, K, ctypes.byref(opt), ctypes.byref(info)), "w4a16_plan")
-    return {name: getattr(info, name) for name, _ in PlanInfo._fields_}
+    return {name: getattr(info, name) for name, _ in PlanInfo._fields_ if name != "reserved"}
 
 
 def w4a16_device_status(stream=None) -> int:

@@ -507,6 +507,61 @@ __device__ __forceinline__ float4 ld_dsmem_f4(uint32_t cluster_addr) {
     return v;
 }
 
+// ------------------------------------------------------------------ L2 prefetch, L2-only loads, DSMEM
+
+// Bring [src, src + bytes) into L2 (bytes a multiple of 16, src 16-byte aligned).  A hint
+// only: L2 is the point of coherence, so prefetching a line that a preceding kernel is
+// still writing is harmless (the write updates the line in L2).
+__device__ __forceinline__ void prefetch_l2_bulk(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+// 128-bit global load through L1 (a plain weak load: after griddepcontrol.wait it sees the
+// preceding kernel's writes).  Four loads of neighbouring 16-byte chunks share their sectors.
+__device__ __forceinline__ uint4 ldg_v4(const void *p) {
+    uint4 v;
+    asm volatile("ld.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+}
+
+// 16-byte store into the shared memory of another CTA of the cluster that completes its
+// bytes on that CTA's mbarrier (complete_tx): no fence, the waiter's phase orders the data.
+__device__ __forceinline__ void st_async_dsmem_f4(uint32_t cluster_addr, float4 v, uint32_t cluster_bar) {
+    asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];"
+                 ::"r"(cluster_addr), "f"(v.x), "f"(v.y), "f"(v.z), "f"(v.w), "r"(cluster_bar)
+                 : "memory");
+}
+
+// Bounded wait with acquire semantics at cluster scope (for phases completed by remote
+// release arrivals).  Same give-up rules as mbar_wait.
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
+    auto test = [&](uint32_t hint) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity), "r"(hint)
+            : "memory");
+        return ok != 0;
+    };
+    if (test(0u)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t spin = 1;; ++spin) {
+        if (test(20000u)) return true;
+        if ((spin & 63u) == 0) {
+            if (status_set()) return false;
+            if (globaltimer() - t0 > kWaitTimeoutNs) {
+                record_timeout();
+                return false;
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ PDL
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }

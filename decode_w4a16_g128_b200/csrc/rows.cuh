@@ -1,36 +1,45 @@
-// rows.cuh - row-block W4A16 matvec for M <= 8 (decode), no split of K across CTAs.
+// rows.cuh - row-block W4A16 matvec for M <= 8 (decode).
 //
 // Role in the layer: tiny-llm "Week 2 Day 6: SIMD-Matrix Prefill", Task 1,
-// keeps a matvec schedule for M <= 8; Task 3 applies one scale and bias per
-// 128-group.  This is a B200 design, not that Metal kernel.
+// keeps a matvec schedule for M <= 8; Task 2 asks for contiguous device loads;
+// Task 3 applies one scale and bias per 128-group; the "Route affine qmv_wide
+// by bit-width and batch size" PR holds a dequantised group in registers and
+// reuses it across the M activation rows.  This is a B200 design, not those
+// Metal kernels.
 //
-// Why a second matvec: in a stream of back-to-back decode projections a call's
-// time is mostly latency (the previous call's completion, x, a cross-CTA
-// fix-up), not bytes.  Here every CTA owns R = 8 n_oct whole weight rows over
-// the whole of K, so no partial sum leaves the CTA, and its codes, scales and
-// biases (at most ~100 KB) are all fetched by TMA / bulk copies at the start.
-// With the static-weights flag that happens before the dependency wait, and
-// since a CTA takes under half of an SM, the next call's CTAs become resident
-// beside this call's and fetch their weights while this one computes.
+// Why this shape: in a stream of back-to-back decode projections a call's time is
+// latency, not bytes, unless the weights are already on chip when the call's
+// input arrives.  So every CTA owns RB row blocks of 16 whole weight rows over a
+// K range, holds ALL of their codes, scales and biases in shared memory (one TMA
+// box of [16 RB rows x 64 B] per 128-group, two copies for scales and biases)
+// and requests them at its start.  With the static-weights flag that happens
+// before the dependency wait; a CTA takes under half of an SM, so the next call's
+// CTAs are resident beside this call's and fetch their weights while this call
+// computes.  Each CTA also prefetches its share of x into L2 before the wait.
+// After the wait only x-dependent work remains: the compute warps load their
+// groups' x straight into registers (all of it in flight at once, two groups of
+// look-ahead), run the MMAs, and the partial sums are added.
 //
-// Layout in shared memory:
-//   codes  ceil(G/2) boxes of [R rows x 128 bytes] (32 code words: two groups),
-//          128-byte swizzle (16-byte chunk c of row r stored at c ^ (r & 7))
-//   scales [R][G] BF16, biases [R][G] BF16 (contiguous rows of the inputs)
-//   after the main loop the codes area holds the compute warps' partial sums
+// Compute: m16n8k16 BF16 tensor-core MMAs with the CODES as A (16 weight rows
+// x 16 k) and x as B (16 k x 8 columns = the M <= 8 activation rows, zeros
+// beyond M), so every MMA row is a real weight row.  Codes enter as the exact
+// BF16 values 128 + q (one LOP3 per two codes); the MMA yields
+// P' = sum (128 + q) x, and the group sum X = sum x comes from MMAs against
+// all-ones A.  The epilogue adds s P' + (b - 128 s) X in FP32 per group.
+// Lane (g, t) = (lane / 4, lane % 4) reads code words 4t .. 4t+3 of rows g and
+// g + 8 of a row block (k = 32t .. 32t+31 of the group, one 16-byte load per
+// row, conflict-free: a quarter warp covers two 64-byte rows) and the same 32 k
+// of x row g.  Word c feeds two MMAs: nibble pairs (0,4),(1,5) and (2,6),(3,7),
+// with x permuted identically (a permutation of k shared by A and B leaves the
+// dot product unchanged).
 //
-// Compute: m16n8k16 BF16 tensor-core MMAs with x as A (16 rows, the M <= 8
-// activation rows then zeros) and the codes as B (16 k x 8 weight rows), one
-// warp per contiguous range of groups.  Codes enter as the exact BF16 values
-// 128 + q; for each group and weight row the MMA yields P' = P + 128 X, with
-// X the group sum of x (from MMAs of x against ones), and the epilogue adds
-// s P' + (b - 128 s) X in FP32.  Per lane (m = lane / 4, t = lane % 4) and
-// group: four code words 4t .. 4t+3 of its weight row and the same 32 k of x
-// row m; word q, nibble pairs (0,4),(1,5) feed MMA 2q and (2,6),(3,7) MMA
-// 2q+1, with x permuted to match (any permutation of k shared by A and B
-// leaves the dot product unchanged).
-//
-// The partial sums of the compute warps are added in warp order (deterministic).
+// Work split: the CTA's (row block, group) units are ordered group-major and cut
+// into 8 contiguous, equal ranges, one per compute warp; the warps' partial sums
+// are added in warp order through shared memory.  Optionally S CTAs of a cluster
+// share the same rows, each a contiguous K range: ranks 1..S-1 store their
+// partials into rank 0's shared memory and arrive on its barrier (release at
+// cluster scope); rank 0 adds them in rank order.  Every sum has a fixed order:
+// the result does not depend on timing.
 #pragma once
 
 #include "ptx.cuh"
@@ -39,35 +48,39 @@ namespace w4a16 {
 namespace mvr {
 
 constexpr int kMaxM = 8;
-constexpr int kComputeWarps = 8;
-constexpr int kThreads = (1 + kComputeWarps) * 32;   // warp 0: producer
-constexpr int kMaxOct = 9;                           // weight-row octets per CTA: R <= 72
-constexpr int kBudget = 110 * 1024;                  // shared memory per CTA: two CTAs per SM
-constexpr uint32_t kBarReduce = 1;                   // named barrier of the compute warps
+constexpr int kWarps = 8;                            // every warp computes; thread 0 also issues the copies
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxRB = 5;                            // row blocks of 16 rows per CTA
+constexpr int kMaxSplits = 4;                        // CTAs of a cluster sharing rows (K split)
+constexpr int kXD = 2;                               // groups of x look-ahead per warp (registers)
+// Shared memory of a CTA: two fit on an SM (233472 B less 1 KB reserved per CTA).
+constexpr long long kBudget = 115712;
+constexpr int kGather = 8;                           // scale / bias loads in flight per thread (K split)
 
-__host__ __device__ constexpr int boxes(int G) { return (G + 1) / 2; }
-__host__ __device__ constexpr long long codes_bytes(int noct, int G) { return 8ll * noct * 128 * boxes(G); }
-__host__ __device__ constexpr long long sb_bytes(int noct, int G) {   // scales or biases, 16-byte rounded
-    return (16ll * noct * G + 15) / 16 * 16;
+// A cluster owns hb blocks of 8 rows ("half blocks"); its MMA row blocks are rb = ceil(hb / 2),
+// the last one half used when hb is odd.  A group's codes take 8 hb rows of 64 B; the MMA of
+// a half-used block also reads the 8 rows after the slot, so the area has 512 B of slack.
+__host__ __device__ constexpr int rbs_of(int hb) { return (hb + 1) / 2; }
+__host__ __device__ constexpr long long codes_bytes(int hb, int gc) { return 512ll * hb * gc + 512; }
+__host__ __device__ constexpr long long red_bytes(int hb) { return 4096ll * rbs_of(hb); }   // [8][rb][16][8] FP32
+__host__ __device__ constexpr long long work_bytes(int hb, int gc) {
+    return codes_bytes(hb, gc) > red_bytes(hb) ? codes_bytes(hb, gc) : red_bytes(hb);
 }
-__host__ __device__ constexpr long long red_bytes(int noct) { return 4ll * kComputeWarps * 8 * noct * kMaxM; }
-__host__ __device__ constexpr long long smem_bytes(int noct, int G) {
-    const long long work = codes_bytes(noct, G) > red_bytes(noct) ? codes_bytes(noct, G) : red_bytes(noct);
-    return work + 2 * sb_bytes(noct, G) + 8ll * (boxes(G) + 1) + 1024;   // + barriers + alignment slack
+// scales or biases [16 rb][gc] BF16 (rows past the half blocks are read, never used)
+__host__ __device__ constexpr long long sb_bytes(int hb, int gc) { return (32ll * rbs_of(hb) * gc + 15) / 16 * 16; }
+__host__ __device__ constexpr long long part_bytes(int hb) { return 512ll * rbs_of(hb); }   // [16 rb][8] FP32
+// work | scales | biases | own partial (S > 1) | partials of ranks 1..S-1 (rank 0) | barriers
+__host__ __device__ constexpr long long off_scales(int hb, int gc) { return work_bytes(hb, gc); }
+__host__ __device__ constexpr long long off_biases(int hb, int gc) { return off_scales(hb, gc) + sb_bytes(hb, gc); }
+__host__ __device__ constexpr long long off_part(int hb, int gc) { return off_biases(hb, gc) + sb_bytes(hb, gc); }
+__host__ __device__ constexpr long long off_slots(int hb, int gc, int s) {
+    return off_part(hb, gc) + (s > 1 ? part_bytes(hb) : 0);
 }
-
-// Octets per CTA for an N x K matrix on `sms` SMs: as few CTAs as cover the rows in
-// one pass, at most two per SM; 0 if no such split fits the budget (the stream-K
-// matvec serves that size).
-__host__ __device__ constexpr int plan_octets(long long N, long long K, int sms) {
-    if (N <= 0 || K <= 0 || sms <= 0) return 0;
-    const long long oct = (N + 7) / 8;
-    const int G = static_cast<int>(K / 128);
-    const long long hi = (oct + sms - 1) / sms;               // one CTA per SM
-    const long long lo = (oct + 2ll * sms - 1) / (2ll * sms);  // two CTAs per SM
-    for (long long n = hi < kMaxOct ? hi : kMaxOct; n >= lo && n >= 1; --n)
-        if (smem_bytes(static_cast<int>(n), G) <= kBudget) return static_cast<int>(n);
-    return 0;
+__host__ __device__ constexpr long long off_bars(int hb, int gc, int s) {
+    return off_slots(hb, gc, s) + (s - 1) * part_bytes(hb);
+}
+__host__ __device__ constexpr long long smem_bytes(int hb, int gc, int s) {
+    return off_bars(hb, gc, s) + 8ll * (gc + 2) + 128;   // + barriers, + alignment slack
 }
 
 struct Params {
@@ -76,151 +89,254 @@ struct Params {
     const uint16_t *biases;   // bf16 [N, G]
     uint16_t *y;              // bf16 [M, N]
     int M, N, K, G;
-    int noct;                 // weight-row octets per CTA (R = 8 noct)
+    int splits;               // S: CTAs of a cluster, each a contiguous run of groups
+    int gcl;                  // ceil(G / S): groups of the shared-memory layout
+    int nh;                   // 8-row half blocks of the matrix, ceil(N / 8)
+    int clusters;             // clusters with rows: cluster c owns half blocks [c nh / clusters, (c+1) nh / clusters)
+    int hb_lo, hb_hi;         // floor / ceil(nh / clusters): tm_lo / tm_hi boxes; 8 hb_hi rows per group slot
     int static_weights;       // codes, scales and biases may be read before the dependency wait
+    long long x_chunk;        // bytes of x this CTA prefetches into L2 (0: none)
 };
 
 // BF16 pair (lo, hi) of two words' low / high halves
 __device__ __forceinline__ uint32_t lo_halves(uint32_t a, uint32_t b) { return prmt(a, b, 0x5410u); }
 __device__ __forceinline__ uint32_t hi_halves(uint32_t a, uint32_t b) { return prmt(a, b, 0x7632u); }
 
-// D += A B with A = x fragment (rows m, m+8: a1 = a3 = 0) and B = (b0, b1); d2, d3 stay 0
-__device__ __forceinline__ void mma_x(float (&d)[4], uint32_t a0, uint32_t a2, uint32_t b0, uint32_t b1) {
-    const uint32_t a[4] = {a0, 0u, a2, 0u};
-    mma_bf16_16816(d, a, b0, b1, d);
+__device__ __forceinline__ void load_x(uint4 (&xr)[4], const uint16_t *src, bool live) {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) xr[q] = live ? ldg_v4(src + 8 * q) : make_uint4(0u, 0u, 0u, 0u);
 }
 
-// Two CTAs per SM: 2 x 288 threads x 112 registers <= 65536.
-__global__ void __maxnreg__(112)
-    rows_kernel(const __grid_constant__ CUtensorMap tm_w, const Params p) {
+// Two CTAs per SM: each SM sub-partition holds 2 + 2 of their warps, 4 x 32 x 128 = 16384 registers.
+template <int RB>
+__global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap tm_hi,
+                                            const __grid_constant__ CUtensorMap tm_lo, const Params p) {
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-    const int G = p.G, noct = p.noct, R = 8 * noct;
-    const int nbox = boxes(G);
-    const long long cbytes = codes_bytes(noct, G) > red_bytes(noct) ? codes_bytes(noct, G) : red_bytes(noct);
-    uint16_t *sc = reinterpret_cast<uint16_t *>(smem + cbytes);
-    uint16_t *bi = reinterpret_cast<uint16_t *>(smem + cbytes + sb_bytes(noct, G));
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + cbytes + 2 * sb_bytes(noct, G));
-    uint64_t *box_full = bars, *sb_full = bars + nbox;
+    uint8_t *smem = smem_raw + ((128u - (smem_u32(smem_raw) & 127u)) & 127u);
+    const int S = p.splits, GCL = p.gcl, G = p.G, HB = p.hb_hi;
+    const int slot = 8 * HB * 64;                                        // bytes of one group's codes
+    const uint32_t rank = S > 1 ? cluster_ctarank() : 0u;
+    // this cluster's row blocks; clusters past p.clusters have none (they keep one CTA of
+    // every call on each SM, so that the next call's CTAs land one per SM)
+    const int cl = static_cast<int>(blockIdx.x) / S;
+    const int hb0 = static_cast<int>(static_cast<long long>(cl) * p.nh / p.clusters);
+    const int nhb = cl < p.clusters ? static_cast<int>(static_cast<long long>(cl + 1) * p.nh / p.clusters) - hb0 : 0;
+    const int nrb = (nhb + 1) / 2;                                       // MMA row blocks (<= RB)
+    const long long r0 = 8ll * hb0;                                      // first weight row of the CTA
+    const int g0 = static_cast<int>(rank * G / S), g1 = static_cast<int>((rank + 1) * G / S);
+    const int GC = g1 - g0;                                              // groups of this CTA
+    uint16_t *sc = reinterpret_cast<uint16_t *>(smem + off_scales(HB, GCL));
+    uint16_t *bi = reinterpret_cast<uint16_t *>(smem + off_biases(HB, GCL));
+    float *part = reinterpret_cast<float *>(smem + off_part(HB, GCL));
+    float *slots = reinterpret_cast<float *>(smem + off_slots(HB, GCL, S));
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + off_bars(HB, GCL, S));
+    uint64_t *box_full = bars, *sb_full = bars + GCL, *red_full = bars + GCL + 1;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const long long r0 = static_cast<long long>(blockIdx.x) * R;   // first weight row of this CTA
 
     if (threadIdx.x == 0) {
         pdl_launch_dependents();   // the next call may start fetching its weights
-        for (int b = 0; b <= nbox; ++b) mbar_init(&bars[b], 1);
+        for (int b = 0; b < GC; ++b) mbar_init(&box_full[b], 1);
+        mbar_init(sb_full, 1);
+        mbar_init(red_full, 1);
+        if (S > 1 && rank == 0)   // the other ranks' partials arrive as bytes on this barrier
+            mbar_arrive_expect_tx(red_full, static_cast<uint32_t>((S - 1) * part_bytes(HB)));
         fence_mbar_init();
     }
-    __syncthreads();
-
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer (one thread)
-        if (lane != 0) return;
-        prefetch_tmap(&tm_w);
-        if (!p.static_weights) pdl_wait();
-        // scales and biases of rows r0 .. r0+R-1: one contiguous [rows][G] block each
-        const long long rows = max(0ll, min(static_cast<long long>(R), p.N - r0));
-        const uint32_t bytes = static_cast<uint32_t>(rows * G * 2);
-        const uint32_t bulk = bytes & ~15u;
-        for (uint32_t e = bulk / 2; e < bytes / 2; ++e) {   // ragged end
-            sc[e] = __ldg(p.scales + r0 * G + e);
-            bi[e] = __ldg(p.biases + r0 * G + e);
-        }
-        mbar_arrive_expect_tx(sb_full, 2 * bulk);
-        if (bulk) {
-            bulk_load(sc, p.scales + r0 * G, bulk, sb_full);
-            bulk_load(bi, p.biases + r0 * G, bulk, sb_full);
-        }
-        // codes: box b = words 32 b .. 32 b + 31 of rows r0 .. r0+R-1 (zeros past N and K)
-        for (int b = 0; b < nbox; ++b) {
-            mbar_arrive_expect_tx(&box_full[b], static_cast<uint32_t>(R) * 128);
-            tma_load_2d(smem + static_cast<long long>(b) * R * 128, &tm_w, &box_full[b], 32 * b, static_cast<int>(r0));
-        }
-        // leave no copy in flight
-        for (int b = 0; b <= nbox; ++b) mbar_wait(&bars[b], 0, /*give_up_on_status=*/false);
+    if (S > 1)
+        cluster_sync_all();   // rank 0's barrier is initialised before any rank can arrive on it
+    else
+        __syncthreads();
+    if (nhb == 0) {           // no rows: hold the slot until the preceding kernel is done
+        pdl_wait();
         return;
     }
 
-    // ---------------------------------------------------------------- compute warps
-    const int w = warp - 1;
-    const int m = lane >> 2, t = lane & 3;   // x row (A row, D row); thread in quad
-    const bool live = m < p.M;
-    const int ga = w * G / kComputeWarps, gb = (w + 1) * G / kComputeWarps;   // this warp's groups
-    float out[kMaxOct][2];
-#pragma unroll
-    for (int o = 0; o < kMaxOct; ++o) out[o][0] = out[o][1] = 0.f;
-    constexpr uint32_t kOnes = 0x3F803F80u;   // BF16 (1.0, 1.0)
-    pdl_wait();   // x may come from the preceding kernel
-    bool ok = ga >= gb || mbar_wait(sb_full, 0);
-    const uint4 *xrow = reinterpret_cast<const uint4 *>(p.x + static_cast<long long>(live ? m : 0) * p.K);
-    uint4 xv[4];
-    if (ok && ga < gb) {
-#pragma unroll
-        for (int q = 0; q < 4; ++q) xv[q] = live ? __ldg(xrow + 16 * ga + 4 * t + q) : make_uint4(0, 0, 0, 0);
-    }
-    const uint32_t cbase = smem_u32(smem);
-    for (int g = ga; ok && g < gb; ++g) {
-        // A fragments of this group (x permuted like the codes), and the next group's x
-        uint32_t a[4][2][2];   // [word q][MMA 2q + h][a0, a2]
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-            a[q][0][0] = lo_halves(xv[q].x, xv[q].z);   // x0, x4
-            a[q][0][1] = hi_halves(xv[q].x, xv[q].z);   // x1, x5
-            a[q][1][0] = lo_halves(xv[q].y, xv[q].w);   // x2, x6
-            a[q][1][1] = hi_halves(xv[q].y, xv[q].w);   // x3, x7
+    // ---------------------------------------------------------------- weights, then the wait
+    if (!p.static_weights) pdl_wait();
+    const long long rows = max(0ll, min(8ll * nhb, p.N - r0));
+    if (threadIdx.x == 0) {
+        const CUtensorMap *tm = nhb == p.hb_lo ? &tm_lo : &tm_hi;   // boxes of 8 nhb rows
+        prefetch_tmap(tm);
+        // codes: box b = words 16 (g0 + b) .. + 15 of rows r0 .. r0 + 8 nhb - 1 (zeros past N)
+        for (int b = 0; b < GC; ++b) {
+            mbar_arrive_expect_tx(&box_full[b], static_cast<uint32_t>(nhb) * 512);
+            tma_load_2d(smem + static_cast<long long>(b) * slot, tm, &box_full[b], 16 * (g0 + b),
+                        static_cast<int>(r0));
         }
-        if (g + 1 < gb) {
-#pragma unroll
-            for (int q = 0; q < 4; ++q) xv[q] = live ? __ldg(xrow + 16 * (g + 1) + 4 * t + q) : make_uint4(0, 0, 0, 0);
-        }
-        // group sum of x row m (every column of D holds it)
-        float xs[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int q = 0; q < 4; ++q)
-#pragma unroll
-            for (int h = 0; h < 2; ++h) mma_x(xs, a[q][h][0], a[q][h][1], kOnes, kOnes);
-        const float X = xs[0];
-        if (((g - ga) == 0 || (g & 1) == 0) && !mbar_wait(&box_full[g >> 1], 0)) { ok = false; break; }
-        // chunk 4 (g % 2) + t of row 8 o + m in box g / 2, swizzled by the row's low bits (= m)
-        const uint32_t cw = cbase + static_cast<uint32_t>(g >> 1) * R * 128 + m * 128 +
-                            ((static_cast<uint32_t>(4 * (g & 1) + t) ^ static_cast<uint32_t>(m)) << 4);
-#pragma unroll
-        for (int o = 0; o < kMaxOct; ++o) {
-            if (o >= noct) break;
-            const uint4 c = lds128(cw + o * 8 * 128);
-            const uint32_t cw4[4] = {c.x, c.y, c.z, c.w};
-            float pa[4] = {0.f, 0.f, 0.f, 0.f}, pb[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                const uint32_t v = cw4[q];
-                mma_x(pa, a[q][0][0], a[q][0][1], codes_to_bf16x2_plus128(v), codes_to_bf16x2_plus128(v >> 4));
-                mma_x(pb, a[q][1][0], a[q][1][1], codes_to_bf16x2_plus128(v >> 8), codes_to_bf16x2_plus128(v >> 12));
+        if (S == 1) {
+            // scales and biases of the CTA's rows: one contiguous [rows][G] block each
+            const uint32_t bytes = static_cast<uint32_t>(rows * G * 2);
+            const uint32_t bulk = bytes & ~15u;
+            for (uint32_t e = bulk / 2; e < bytes / 2; ++e) {   // ragged end
+                sc[e] = __ldg(p.scales + r0 * G + e);
+                bi[e] = __ldg(p.biases + r0 * G + e);
             }
-            // weight rows 8 o + 2 t, 8 o + 2 t + 1 of this CTA
-            const int n0 = 8 * o + 2 * t;
-            const float s0 = bf16_to_f32(sc[n0 * G + g]), s1 = bf16_to_f32(sc[(n0 + 1) * G + g]);
-            const float b0 = fmaf(-128.f, s0, bf16_to_f32(bi[n0 * G + g]));
-            const float b1 = fmaf(-128.f, s1, bf16_to_f32(bi[(n0 + 1) * G + g]));
-            out[o][0] = fmaf(b0, X, fmaf(s0, pa[0] + pb[0], out[o][0]));
-            out[o][1] = fmaf(b1, X, fmaf(s1, pa[1] + pb[1], out[o][1]));
+            mbar_arrive_expect_tx(sb_full, 2 * bulk);
+            if (bulk) {
+                bulk_load(sc, p.scales + r0 * G, bulk, sb_full);
+                bulk_load(bi, p.biases + r0 * G, bulk, sb_full);
+            }
+        } else {
+            mbar_arrive(sb_full);   // gathered below, ordered by the CTA barrier
+        }
+        // this CTA's share of x into L2, ahead of the dependency wait
+        if (p.x_chunk > 0) {
+            const long long total = static_cast<long long>(p.M) * p.K * 2;
+            const long long start = static_cast<long long>(blockIdx.x) * p.x_chunk;
+            if (start < total)
+                prefetch_l2_bulk(reinterpret_cast<const uint8_t *>(p.x) + start,
+                                 static_cast<uint32_t>(min(p.x_chunk, total - start)));
         }
     }
-    // ---------------------------------------------------------------- fixed-order sum over warps
-    named_bar_sync(kBarReduce, kComputeWarps * 32);   // every warp is done with the codes
-    float *red = reinterpret_cast<float *>(smem);     // [warp][row n < R][x row m < 8]
+    if (S > 1) {
+        // a K range of the rows, [rows][GC] out of [N][G] (not a contiguous block and not
+        // 16-byte aligned): every thread keeps kGather loads of each array in flight
+        const int n = static_cast<int>(rows) * GC;
+        for (int base = 0; base < n; base += kThreads * kGather) {
+            uint16_t vs[kGather], vb[kGather];
 #pragma unroll
-    for (int o = 0; o < kMaxOct; ++o) {
-        if (o >= noct) break;
-        const int n0 = 8 * o + 2 * t;
-        red[(w * R + n0) * kMaxM + m] = out[o][0];
-        red[(w * R + n0 + 1) * kMaxM + m] = out[o][1];
+            for (int j = 0; j < kGather; ++j) {
+                const int i = base + j * kThreads + static_cast<int>(threadIdx.x);
+                if (i < n) {
+                    const int r = i / GC, c = i - r * GC;
+                    const long long src = (r0 + r) * G + g0 + c;
+                    vs[j] = __ldg(p.scales + src);
+                    vb[j] = __ldg(p.biases + src);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < kGather; ++j) {
+                const int i = base + j * kThreads + static_cast<int>(threadIdx.x);
+                if (i < n) {
+                    const int r = i / GC, c = i - r * GC;
+                    sc[r * GCL + c] = vs[j];
+                    bi[r * GCL + c] = vb[j];
+                }
+            }
+        }
+        __syncthreads();
     }
-    named_bar_sync(kBarReduce, kComputeWarps * 32);
-    for (int i = threadIdx.x - 32; i < R * p.M; i += kComputeWarps * 32) {
-        const int n = i / p.M, mm = i - n * p.M;
+
+    // ---------------------------------------------------------------- compute
+    const int w = warp;
+    const int g = lane >> 2, t = lane & 3;
+    const int U = nrb * GC;                       // units (row block, group), group-major
+    const int u0 = w * U / kWarps, u1 = (w + 1) * U / kWarps;
+    float out[RB][4];
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) out[rb][0] = out[rb][1] = out[rb][2] = out[rb][3] = 0.f;
+    constexpr uint32_t kOnes = 0x3F803F80u;       // BF16 (1.0, 1.0)
+    const uint32_t ones[4] = {kOnes, kOnes, kOnes, kOnes};
+    if (p.static_weights) pdl_wait();             // x may come from the preceding kernel
+    if (u0 < u1) {
+        const int ga = u0 / nrb, gb = (u1 - 1) / nrb + 1;   // groups [ga, gb) of the CTA's range
+        const bool live = g < p.M;
+        const uint16_t *xrow = p.x + static_cast<long long>(live ? g : 0) * p.K + static_cast<long long>(g0) * 128 + 32 * t;
+        uint4 xr[kXD][4];
+#pragma unroll
+        for (int j = 0; j < kXD; ++j)
+            if (ga + j < gb) load_x(xr[j], xrow + (ga + j) * 128, live);
+        bool ok = mbar_wait(sb_full, 0);
+        const uint32_t cbase = smem_u32(smem) + static_cast<uint32_t>(g * 64 + t * 16);
+        for (int gi = ga; ok && gi < gb; gi += kXD) {
+#pragma unroll
+            for (int j = 0; j < kXD; ++j) {
+                const int gg = gi + j;
+                if (gg >= gb) break;
+                // B fragments of group gg (x permuted like the codes), then the next x loads
+                uint32_t bf[8][2];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    bf[2 * c][0] = lo_halves(xr[j][c].x, xr[j][c].z);       // x0, x4
+                    bf[2 * c][1] = hi_halves(xr[j][c].x, xr[j][c].z);       // x1, x5
+                    bf[2 * c + 1][0] = lo_halves(xr[j][c].y, xr[j][c].w);   // x2, x6
+                    bf[2 * c + 1][1] = hi_halves(xr[j][c].y, xr[j][c].w);   // x3, x7
+                }
+                if (gg + kXD < gb) load_x(xr[j], xrow + (gg + kXD) * 128, live);
+                // group sums of x rows 2t, 2t + 1 (two independent MMA chains)
+                float xa[4] = {0.f, 0.f, 0.f, 0.f}, xb[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    mma_bf16_16816(xa, ones, bf[2 * c][0], bf[2 * c][1], xa);
+                    mma_bf16_16816(xb, ones, bf[2 * c + 1][0], bf[2 * c + 1][1], xb);
+                }
+                const float X0 = xa[0] + xb[0], X1 = xa[1] + xb[1];
+                if (!mbar_wait(&box_full[gg], 0)) { ok = false; break; }
+                const int rlo = gg == ga ? u0 - ga * nrb : 0;
+                const int rhi = gg == gb - 1 ? u1 - gg * nrb : nrb;
+                const uint32_t cg = cbase + static_cast<uint32_t>(gg * slot);
+#pragma unroll
+                for (int rb = 0; rb < RB; ++rb) {
+                    if (rb < rlo || rb >= rhi) continue;
+                    // words 4t .. 4t + 3 of rows 16 rb + g and 16 rb + g + 8, group gg
+                    const uint4 ca = lds128(cg + rb * 16 * 64), cb = lds128(cg + rb * 16 * 64 + 8 * 64);
+                    const uint32_t wa[4] = {ca.x, ca.y, ca.z, ca.w}, wb[4] = {cb.x, cb.y, cb.z, cb.w};
+                    float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const uint32_t a0[4] = {codes_to_bf16x2_plus128(wa[c]), codes_to_bf16x2_plus128(wb[c]),
+                                                codes_to_bf16x2_plus128(wa[c] >> 4), codes_to_bf16x2_plus128(wb[c] >> 4)};
+                        mma_bf16_16816(da, a0, bf[2 * c][0], bf[2 * c][1], da);
+                        const uint32_t a1[4] = {codes_to_bf16x2_plus128(wa[c] >> 8), codes_to_bf16x2_plus128(wb[c] >> 8),
+                                                codes_to_bf16x2_plus128(wa[c] >> 12), codes_to_bf16x2_plus128(wb[c] >> 12)};
+                        mma_bf16_16816(db, a1, bf[2 * c + 1][0], bf[2 * c + 1][1], db);
+                    }
+                    // scale and shifted bias of rows 16 rb + g (A row g) and 16 rb + g + 8 (A row g + 8)
+                    const int na = (rb * 16 + g) * GCL + gg, nb = na + 8 * GCL;
+                    const float sa = bf16_to_f32(sc[na]), sb = bf16_to_f32(sc[nb]);
+                    const float ba = fmaf(-128.f, sa, bf16_to_f32(bi[na]));
+                    const float bb = fmaf(-128.f, sb, bf16_to_f32(bi[nb]));
+                    out[rb][0] = fmaf(ba, X0, fmaf(sa, da[0] + db[0], out[rb][0]));
+                    out[rb][1] = fmaf(ba, X1, fmaf(sa, da[1] + db[1], out[rb][1]));
+                    out[rb][2] = fmaf(bb, X0, fmaf(sb, da[2] + db[2], out[rb][2]));
+                    out[rb][3] = fmaf(bb, X1, fmaf(sb, da[3] + db[3], out[rb][3]));
+                }
+            }
+        }
+    }
+    // ---------------------------------------------------------------- fixed-order sums
+    __syncthreads();   // every warp is done with the codes
+    float *red = reinterpret_cast<float *>(smem);   // [warp][row block][row][x row]
+#pragma unroll
+    for (int rb = 0; rb < RB; ++rb) {
+        float *dst = red + ((w * RB + rb) * 16 + g) * kMaxM + 2 * t;
+        *reinterpret_cast<float2 *>(dst) = make_float2(out[rb][0], out[rb][1]);
+        *reinterpret_cast<float2 *>(dst + 8 * kMaxM) = make_float2(out[rb][2], out[rb][3]);
+    }
+    __syncthreads();
+    const int tid = threadIdx.x;
+    const int RC = 8 * nhb;                      // rows of this CTA
+    const int RM = RC * p.M;
+    for (int i = tid; i < RM; i += kWarps * 32) {
+        const int m = i / RC, r = i - m * RC;
+        const float *src = red + r * kMaxM + m;   // row block r / 16, row r % 16: offset r * 8
         float v = 0.f;
 #pragma unroll
-        for (int ww = 0; ww < kComputeWarps; ++ww) v += red[(ww * R + n) * kMaxM + mm];
-        if (r0 + n < p.N) p.y[static_cast<long long>(mm) * p.N + r0 + n] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        for (int ww = 0; ww < kWarps; ++ww) v += src[ww * RB * 16 * kMaxM];
+        if (S == 1) {
+            if (r0 + r < p.N) p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        } else {
+            part[r * kMaxM + m] = v;
+        }
+    }
+    if (S == 1) return;
+    // ---------------------------------------------------------------- K split over the cluster
+    if (rank != 0) {
+        // this CTA's partial into slot rank - 1 of rank 0: asynchronous remote stores whose
+        // bytes complete on rank 0's barrier
+        __syncthreads();
+        const uint32_t dst = dsmem_addr(smem_u32(slots + (rank - 1) * 16 * RB * kMaxM), 0u);
+        const uint32_t bar = dsmem_addr(smem_u32(red_full), 0u);
+        for (int i = tid; i < 16 * RB * kMaxM / 4; i += kWarps * 32)
+            st_async_dsmem_f4(dst + 16u * i, reinterpret_cast<const float4 *>(part)[i], bar);
+        return;
+    }
+    const bool ok = mbar_wait_cluster(red_full, 0);
+    for (int i = tid; ok && i < RM; i += kWarps * 32) {
+        const int m = i / RC, r = i - m * RC;
+        float v = part[r * kMaxM + m];
+        for (int s = 1; s < S; ++s) v += slots[((s - 1) * 16 * RB + r) * kMaxM + m];
+        if (r0 + r < p.N) p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
     }
 }
 

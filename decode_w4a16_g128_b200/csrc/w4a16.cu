@@ -61,6 +61,25 @@ std::mutex g_mu;
 std::map<int, DeviceInfo> g_devices;
 std::map<std::pair<int, void *>, Workspace> g_workspaces;
 
+template <int RB>
+cudaError_t rows_set_attributes_one() {
+    cudaError_t e = cudaFuncSetAttribute(mvr::rows_kernel<RB>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(mvr::kBudget));
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(mvr::rows_kernel<RB>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    return e;
+}
+
+cudaError_t rows_set_attributes() {
+    static_assert(mvr::kMaxRB == 5, "one instantiation per row-block count");
+    cudaError_t e = rows_set_attributes_one<1>();
+    if (e == cudaSuccess) e = rows_set_attributes_one<2>();
+    if (e == cudaSuccess) e = rows_set_attributes_one<3>();
+    if (e == cudaSuccess) e = rows_set_attributes_one<4>();
+    if (e == cudaSuccess) e = rows_set_attributes_one<5>();
+    return e;
+}
+
 // Per-device one-time set-up: capability check, SM count, driver entry point,
 // kernel attributes.  Caller holds g_mu.
 int device_setup(int dev, DeviceInfo **out) {
@@ -87,11 +106,9 @@ int device_setup(int dev, DeviceInfo **out) {
             if (e != cudaSuccess) return cuda_fail(e);
             d.gemm_ok = fa.numRegs * gm::kThreads >=
                         128 * (gm::kRegsCtl + 2 * gm::kRegsDeq + 2 * gm::kRegsEpi);
-            e = cudaFuncSetAttribute(mvr::rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, mvr::kBudget);
-            // the largest shared-memory carveout: two CTAs per SM (without it the driver
-            // picks a split that holds one), and the same split as the other kernels
-            if (e == cudaSuccess)
-                e = cudaFuncSetAttribute(mvr::rows_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+            // the largest shared-memory carveout: two row-block CTAs per SM (without it the
+            // driver picks a split that holds one), and the same split as the other kernels
+            e = rows_set_attributes();
             if (e != cudaSuccess) return cuda_fail(e);
             e = cudaFuncSetAttribute(mv::matvec_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      int(kMatvecBudget));
@@ -250,7 +267,8 @@ int choose_path(int64_t M, const w4a16_options *opt, int *path) {
 
 int validate_options(const w4a16_options *opt) {
     if (!opt) return W4A16_OK;
-    if (opt->splits < 0 || opt->splits > gm::kMaxSplits || opt->workers < 0 || opt->sm_count < 0)
+    if (opt->splits < 0 || opt->splits > gm::kMaxSplits || opt->workers < 0 || opt->sm_count < 0 ||
+        opt->row_blocks < 0 || opt->row_blocks > mvr::kMaxRB)
         return W4A16_ERR_INVALID_ARG;
     if (opt->flags & ~(W4A16_FLAG_NO_PDL | W4A16_FLAG_STATIC_WEIGHTS)) return W4A16_ERR_INVALID_ARG;
     return W4A16_OK;
@@ -351,21 +369,79 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
     pl->workspace_bytes = (M + N) * gm::xs_cols(static_cast<int>(G)) * 2;   // bias-step operands
 }
 
-// Row-block matvec: ceil(N / (8 noct)) CTAs of 8 noct whole weight rows each.
-void plan_rows(int64_t N, int64_t K, int noct, w4a16_plan_info *pl) {
-    const int64_t oct = (N + 7) / 8;
-    const int64_t grid = (oct + noct - 1) / noct;
-    noct = static_cast<int>((oct + grid - 1) / grid);   // the same CTA count may need fewer octets each
+// Row-block matvec: clusters of S CTAs share blocks of 8 whole weight rows ("half blocks",
+// MMA row blocks of 16 rows, the last one half used for an odd count), each CTA of a cluster
+// a contiguous run of ceil(G / S) or floor(G / S) groups.  The half blocks are spread evenly
+// over at most SMs / S clusters, and the grid is padded with empty clusters to one CTA per
+// SM: every call then holds exactly one CTA on each SM, so the next call's CTAs (resident
+// beside it, fetching their weights) land one per SM too and no SM computes two CTAs of the
+// same call.  The K split is the smallest S (1, 2, 4) whose layout fits and leaves every
+// compute warp at least kRowsMinUnits units (16 rows x one group), else 2 if it fits, else the
+// smallest that fits: measured on B200 in a back-to-back stream of the seven Qwen3-4B decode
+// projections, a split pays for its exchange of partial sums (distributed shared memory) only
+// when the warps have little work (k/v: 2.5 units per warp without a split) or when nothing
+// smaller fits (the 9728-deep projection); clusters of four pack badly beside the next call's
+// CTAs.  A CTA's shared memory leaves room for the next call's.
+constexpr int kRowsMinUnits = 4;
+
+struct RowsChoice {
+    int hb = 0, splits = 0;    // half blocks of the fullest cluster, K splits
+    int64_t clusters = 0;      // clusters with rows
+    int64_t grid = 0;          // CTAs launched (clusters with rows, padded)
+};
+
+bool rows_choose(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, RowsChoice *out) {
+    (void)M;
+    const int64_t NH = (N + 7) / 8, G = K / 128;
+    const int req_rb = opt ? opt->row_blocks : 0, req_s = opt ? opt->splits : 0;
+    const int order[3] = {1, 2, 4};
+    RowsChoice fits[3];
+    int64_t units[3] = {0, 0, 0};
+    int nfit = 0;
+    for (int i = 0; i < 3; ++i) {
+        const int s = req_s ? (i == 0 ? req_s : 0) : order[i];
+        if (s == 0 || s > G) continue;
+        const int64_t gcl = (G + s - 1) / s;
+        const int64_t slots = std::max<int64_t>(1, sms / s);      // clusters that fit one CTA per SM
+        const int64_t clusters = req_rb ? (NH + 2 * req_rb - 1) / (2 * req_rb) : std::min<int64_t>(slots, NH);
+        const int64_t hb = (NH + clusters - 1) / clusters;
+        if (mvr::rbs_of(static_cast<int>(std::min<int64_t>(hb, 1 << 20))) > mvr::kMaxRB) continue;
+        if (mvr::smem_bytes(static_cast<int>(hb), static_cast<int>(std::min<int64_t>(gcl, 1 << 20)), s) > mvr::kBudget)
+            continue;
+        const int64_t grid = std::max(clusters, slots) * s;
+        if (grid > (int64_t(1) << 31) - 1) continue;
+        fits[nfit].hb = static_cast<int>(hb);
+        fits[nfit].splits = s;
+        fits[nfit].clusters = clusters;
+        fits[nfit].grid = grid;
+        units[nfit] = mvr::rbs_of(static_cast<int>(hb)) * gcl / mvr::kWarps;   // units per warp
+        ++nfit;
+    }
+    if (nfit == 0) return false;
+    // the smallest split that leaves the warps enough work; if none does, two (when it fits)
+    int pick = -1;
+    for (int i = 0; i < nfit && pick < 0; ++i)
+        if (units[i] >= kRowsMinUnits) pick = i;
+    for (int i = 0; i < nfit && pick < 0; ++i)
+        if (fits[i].splits == 2) pick = i;
+    if (pick < 0) pick = 0;
+    *out = fits[pick];
+    return true;
+}
+
+void plan_rows(int64_t N, int64_t K, const RowsChoice &c, w4a16_plan_info *pl) {
+    const int64_t G = K / 128;
     std::memset(pl, 0, sizeof(*pl));
     pl->path = W4A16_PATH_MATVEC_ROWS;
-    pl->splits = 1;
-    pl->grid_x = static_cast<int32_t>(grid);
+    pl->splits = c.splits;
+    pl->grid_x = static_cast<int32_t>(c.grid);
     pl->grid_y = pl->grid_z = 1;
     pl->block = mvr::kThreads;
-    pl->smem_bytes = static_cast<int32_t>(mvr::smem_bytes(noct, static_cast<int>(K / 128)));
-    pl->cluster = 1;
-    pl->tiles = pl->grid_x;   // row blocks
-    pl->units = oct;          // weight-row octets
+    pl->smem_bytes = static_cast<int32_t>(mvr::smem_bytes(c.hb, static_cast<int>((G + c.splits - 1) / c.splits), c.splits));
+    pl->cluster = c.splits;
+    pl->tiles = c.clusters;          // clusters with rows
+    pl->units = (N + 7) / 8;         // 8-row half blocks
+    pl->row_blocks = mvr::rbs_of(c.hb);   // MMA row blocks of 16 rows of the fullest cluster
     pl->workspace_bytes = 0;
 }
 
@@ -374,12 +450,14 @@ int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a
     int rc = choose_path(M, opt, &path);
     if (rc) return rc;
     const int req = opt ? opt->path : W4A16_PATH_AUTO;
-    const int noct = mvr::plan_octets(N, K, sms);
-    if (path == W4A16_PATH_MATVEC_ROWS && noct == 0) return W4A16_ERR_UNSUPPORTED;
-    if (path == W4A16_PATH_MATVEC && req == W4A16_PATH_AUTO && !(opt && opt->workers > 0) && noct > 0)
+    RowsChoice rc_rows;
+    const bool rows_fit = path == W4A16_PATH_MATVEC_ROWS || path == W4A16_PATH_MATVEC
+                              ? rows_choose(M, N, K, sms, opt, &rc_rows) : false;
+    if (path == W4A16_PATH_MATVEC_ROWS && !rows_fit) return W4A16_ERR_UNSUPPORTED;
+    if (path == W4A16_PATH_MATVEC && req == W4A16_PATH_AUTO && !(opt && opt->workers > 0) && rows_fit)
         path = W4A16_PATH_MATVEC_ROWS;
     if (path == W4A16_PATH_MATVEC_ROWS) {
-        plan_rows(N, K, noct, pl);
+        plan_rows(N, K, rc_rows, pl);
         return W4A16_OK;
     }
     if (path == W4A16_PATH_MATVEC) {
@@ -412,14 +490,30 @@ int encode_2d(DeviceInfo *d, CUtensorMap *map, CUtensorMapDataType type, const v
     return W4A16_OK;
 }
 
+template <int RB>
+cudaError_t rows_launch_rb(const cudaLaunchConfig_t &cfg, const CUtensorMap &tm_hi, const CUtensorMap &tm_lo,
+                           const mvr::Params &kp) {
+    return cudaLaunchKernelEx(&cfg, mvr::rows_kernel<RB>, tm_hi, tm_lo, kp);
+}
+
 int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void *stream, bool pdl,
                 bool static_weights) {
     const int G = static_cast<int>(p.K / 128);
-    const int noct = static_cast<int>((pl.units + pl.grid_x - 1) / pl.grid_x);
-    CUtensorMap tm_w;
-    // codes: [N, K/8] uint32, boxes of 32 words (128 B: two groups) x 8 noct rows, 128-byte swizzle
-    int rc = encode_2d(d, &tm_w, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 32,
-                       static_cast<uint32_t>(8 * noct), CU_TENSOR_MAP_SWIZZLE_128B);
+    const int rb = pl.row_blocks, S = pl.splits;
+    if (rb < 1 || rb > mvr::kMaxRB || S < 1 || S > mvr::kMaxSplits) return W4A16_ERR_INVALID_ARG;
+    const int64_t NH = (p.N + 7) / 8;
+    const int clusters = static_cast<int>(pl.tiles);
+    const int hb_lo = static_cast<int>(NH / clusters), hb_hi = static_cast<int>((NH + clusters - 1) / clusters);
+    if (mvr::rbs_of(hb_hi) != rb) return W4A16_ERR_INVALID_ARG;
+    CUtensorMap tm_hi, tm_lo;
+    // codes: [N, K/8] uint32, boxes of one group (16 words = 64 B) x the cluster's rows (8 hb_hi,
+    // or 8 hb_lo for the clusters with one half block less), no swizzle (a quarter warp reads
+    // two 64-byte rows: 8 distinct 16-byte bank groups)
+    int rc = encode_2d(d, &tm_hi, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16,
+                       static_cast<uint32_t>(8 * hb_hi), CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (rc) return rc;
+    rc = encode_2d(d, &tm_lo, CU_TENSOR_MAP_DATA_TYPE_UINT32, p.wq, p.K / 8, p.N, p.K / 2, 16,
+                   static_cast<uint32_t>(8 * hb_lo), CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
     mvr::Params kp;
     kp.x = static_cast<const uint16_t *>(p.x);
@@ -430,19 +524,45 @@ int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void
     kp.N = static_cast<int>(p.N);
     kp.K = static_cast<int>(p.K);
     kp.G = G;
-    kp.noct = noct;
+    kp.splits = S;
+    kp.gcl = (G + S - 1) / S;
+    kp.nh = static_cast<int>(NH);
+    kp.clusters = clusters;
+    kp.hb_lo = hb_lo;
+    kp.hb_hi = hb_hi;
     kp.static_weights = static_weights ? 1 : 0;
+    // every CTA prefetches an equal 16-byte-aligned share of x into L2 before the wait
+    const long long xbytes = p.M * p.K * 2;
+    kp.x_chunk = std::min<long long>(((xbytes + pl.grid_x - 1) / pl.grid_x + 15) / 16 * 16, 65536);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(pl.grid_x, 1, 1);
     cfg.blockDim = dim3(pl.block, 1, 1);
     cfg.dynamicSmemBytes = pl.smem_bytes;
     cfg.stream = static_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchAttribute attr[2];
+    int na = 0;
+    if (S > 1) {
+        attr[na].id = cudaLaunchAttributeClusterDimension;
+        attr[na].val.clusterDim.x = S;
+        attr[na].val.clusterDim.y = 1;
+        attr[na].val.clusterDim.z = 1;
+        ++na;
+    }
+    if (pdl) {
+        attr[na].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[na].val.programmaticStreamSerializationAllowed = 1;
+        ++na;
+    }
     cfg.attrs = attr;
-    cfg.numAttrs = pdl ? 1 : 0;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, mvr::rows_kernel, tm_w, kp);
+    cfg.numAttrs = na;
+    cudaError_t e = cudaErrorInvalidValue;
+    switch (rb) {
+        case 1: e = rows_launch_rb<1>(cfg, tm_hi, tm_lo, kp); break;
+        case 2: e = rows_launch_rb<2>(cfg, tm_hi, tm_lo, kp); break;
+        case 3: e = rows_launch_rb<3>(cfg, tm_hi, tm_lo, kp); break;
+        case 4: e = rows_launch_rb<4>(cfg, tm_hi, tm_lo, kp); break;
+        case 5: e = rows_launch_rb<5>(cfg, tm_hi, tm_lo, kp); break;
+    }
     return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 

@@ -65,11 +65,13 @@ enum w4a16_path {
     W4A16_PATH_AUTO = 0,        /* M <= 8: matvec; M > 8: tensor-core GEMM (Task 1 dispatch rule) */
     W4A16_PATH_MATVEC = 1,      /* weight-streaming matvec, M <= 8 only                           */
     W4A16_PATH_GEMM = 2,        /* tcgen05 tensor-core GEMM, any M >= 1                            */
-    W4A16_PATH_MATVEC_ROWS = 3  /* row-block matvec, M <= 8: each CTA owns whole weight rows over all
-                                   of K (no cross-CTA sum), at most two CTAs per SM; only where such
-                                   a split fits (else W4A16_ERR_UNSUPPORTED).  W4A16_PATH_AUTO takes
-                                   it for M <= 8 when it fits and no worker count is given, the
-                                   stream-K matvec (W4A16_PATH_MATVEC) otherwise                   */
+    W4A16_PATH_MATVEC_ROWS = 3  /* row-block matvec, M <= 8: a CTA holds all codes, scales and biases
+                                   of 16 x row_blocks weight rows over a K range in shared memory
+                                   (the whole of K, or 1/splits of it with the splits of a row range
+                                   added in a thread-block cluster); two CTAs fit on an SM.  Only
+                                   where such a split fits (else W4A16_ERR_UNSUPPORTED).
+                                   W4A16_PATH_AUTO takes it for M <= 8 when it fits and no worker
+                                   count is given, the stream-K matvec (W4A16_PATH_MATVEC) otherwise */
 };
 
 /*
@@ -97,12 +99,16 @@ int w4a16_matmul_last_rows(const void *x, const uint32_t *wq, const void *scales
 
 /* Options for the explicit entry points; zero-initialised means "automatic". */
 typedef struct w4a16_options {
-    int32_t path;      /* enum w4a16_path                                                  */
-    int32_t splits;    /* GEMM: K splits (1..4), each a contiguous run of 128-groups; 0 = auto */
-    int32_t workers;   /* matvec: persistent CTAs sharing the (row-tile x group) units; 0 = auto */
-    int32_t sm_count;  /* w4a16_plan only: SM count to plan for; 0 = query the current device   */
-    int32_t flags;     /* W4A16_FLAG_* bits                                                 */
-    int32_t reserved[3];
+    int32_t path;       /* enum w4a16_path                                                  */
+    int32_t splits;     /* GEMM and row-block matvec: K splits (1..4), each a contiguous run of
+                           128-groups; 0 = auto                                              */
+    int32_t workers;    /* stream-K matvec: persistent CTAs sharing the (row-tile x group) units;
+                           0 = auto                                                          */
+    int32_t sm_count;   /* w4a16_plan only: SM count to plan for; 0 = query the current device */
+    int32_t flags;      /* W4A16_FLAG_* bits                                                 */
+    int32_t row_blocks; /* row-block matvec: blocks of 16 weight rows per CTA (1..5); 0 = auto.
+                           With both row_blocks and splits given, that exact launch is used. */
+    int32_t reserved[2];
 } w4a16_options;
 
 /*
@@ -131,16 +137,19 @@ int w4a16_matmul_ex(const void *x, const uint32_t *wq, const void *scales,
 /* What a call of the given size would launch (host-side planning only). */
 typedef struct w4a16_plan_info {
     int32_t path;            /* enum w4a16_path chosen                                  */
-    int32_t splits;          /* GEMM K splits (a cluster holds 2 x splits CTAs); 1 for the matvec */
+    int32_t splits;          /* K splits: GEMM (a cluster holds 2 x splits CTAs) or row-block
+                                matvec (a cluster holds splits CTAs); 1 for the stream-K matvec */
     int32_t grid_x, grid_y, grid_z;   /* GEMM without a K split: a persistent grid of at most
                                          one CTA pair per two SMs, each pair looping over tiles */
     int32_t block;           /* threads per CTA                                         */
     int32_t smem_bytes;      /* dynamic shared memory per CTA                           */
     int32_t cluster;         /* CTAs per cluster (1 = no cluster)                       */
-    int64_t tiles;           /* output tiles (row-block matvec: row blocks, one per CTA) */
+    int64_t tiles;           /* output tiles (row-block matvec: clusters of row_blocks x 16 rows) */
     int64_t units;           /* stream-K matvec: (row tile x 128-group) work units;
-                                row-block matvec: weight-row octets                     */
+                                row-block matvec: 16-row blocks                         */
     int64_t workspace_bytes; /* library workspace the call needs                        */
+    int32_t row_blocks;      /* row-block matvec: blocks of 16 weight rows per cluster   */
+    int32_t reserved;
 } w4a16_plan_info;
 
 /*

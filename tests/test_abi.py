@@ -106,19 +106,35 @@ def test_dispatch_rule():
     assert w4.w4a16_plan(9, 4096, 2560, sm_count=148)["path"] == w4.PATH_GEMM
 
 
-@pytest.mark.parametrize("N,K,noct,grid", [(1024, 2560, 1, 128), (4096, 2560, 4, 128), (2560, 4096, 3, 107),
-                                           (9728, 2560, 9, 136), (2560, 9728, 2, 160), (1000, 256, 1, 125),
-                                           (8, 128, 1, 1), (1, 128, 1, 1)])
-def test_rows_plan(N, K, noct, grid):
-    """Row-block matvec: CTAs of 8 noct whole weight rows, as few as one pass needs, at most
-    two per SM, each within 110 KB of shared memory so that two fit on an SM."""
+def rows_smem(hb, gcl, s):
+    """Shared memory of a row-block CTA: codes of hb half blocks (8 rows) per group plus 512 B
+    of slack (or the warps' partial sums if larger), scales, biases, the cluster's partial sums
+    (own + ranks 1..S-1 on rank 0 when split), barriers, alignment slack."""
+    rb = (hb + 1) // 2
+    work = max(512 * hb * gcl + 512, 4096 * rb)
+    sb = (32 * rb * gcl + 15) // 16 * 16
+    part = 512 * rb * s if s > 1 else 0
+    return work + 2 * sb + part + 8 * (gcl + 2) + 128
+
+
+@pytest.mark.parametrize("N,K,splits", [(1024, 2560, 2), (4096, 2560, 1), (2560, 4096, 1), (9728, 2560, 1),
+                                        (2560, 9728, 2), (1000, 256, 2), (8, 128, 1), (1, 128, 1)])
+def test_rows_plan(N, K, splits):
+    """Row-block matvec: one CTA per SM (padded with CTAs that own no rows), the 8-row half
+    blocks spread evenly over the clusters of `splits` CTAs, at most 5 MMA row blocks of 16
+    rows per cluster, shared memory that leaves room for a second CTA on the SM."""
     pl = w4.w4a16_plan(1, N, K, sm_count=148)
     assert pl["path"] == w4.PATH_MATVEC_ROWS
-    assert pl["block"] == 288            # producer warp + 8 compute warps
-    assert pl["units"] == -(-N // 8)     # weight-row octets
-    assert pl["grid_x"] == grid == -(-pl["units"] // noct)
-    assert pl["grid_x"] <= 2 * 148
-    assert pl["smem_bytes"] <= 110 * 1024 and 2 * (pl["smem_bytes"] + 1024) <= 228 * 1024
+    assert pl["block"] == 256            # 8 warps, all computing
+    assert pl["splits"] == pl["cluster"] == splits
+    nh, G = -(-N // 8), K // 128
+    assert pl["units"] == nh             # 8-row half blocks
+    assert pl["tiles"] == min(148 // splits, nh)
+    assert pl["grid_x"] == (148 // splits) * splits
+    hb = -(-nh // pl["tiles"])
+    assert pl["row_blocks"] == (hb + 1) // 2 <= 5
+    assert pl["smem_bytes"] == rows_smem(hb, -(-G // splits), splits)
+    assert 2 * (pl["smem_bytes"] + 1024) <= 233472
     assert pl["workspace_bytes"] == 0
 
 
@@ -130,27 +146,39 @@ def test_rows_plan_limits():
     with pytest.raises(w4.W4A16Error) as e:
         w4.w4a16_plan(9, 4096, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148)
     assert e.value.status == w4.ERR_UNSUPPORTED
-    # the chosen split: as few CTAs as possible; one octet more per CTA would exceed 110 KB
-    def smem(noct, G):   # codes boxes (or the warps' partial sums), scales, biases, barriers, slack
-        boxes = (G + 1) // 2
-        work = max(8 * noct * 128 * boxes, 4 * 8 * 8 * noct * 8)
-        return work + 2 * ((16 * noct * G + 15) // 16 * 16) + 8 * (boxes + 1) + 1024
-    # 9 octets on 2 SMs, K = 5376: 5 octets per CTA exceed 110 KB, 4 fit, and the 3 CTAs
-    # that 4 octets need hold 3 octets each: the plan describes what is launched
-    pl = w4.w4a16_plan(1, 72, 5376, path=w4.PATH_MATVEC_ROWS, sm_count=2)
-    assert smem(5, 42) > 110 * 1024 >= smem(4, 42)
-    assert pl["grid_x"] == 3 and pl["smem_bytes"] == smem(3, 42)
+    # K = 9728 without a split would need 2 row blocks x 76 groups: more than half an SM
+    assert rows_smem(4, 76, 1) > 115712 >= rows_smem(5, 38, 2)
+    # every plan the rule produces: one CTA per SM, the fewest splits that fit with enough
+    # work per warp (at least 4 units of 16 rows x one group), else 2, else the fewest that fit
     for N in (8, 100, 1000, 2560, 4096, 9728, 20000):
         for K in (128, 256, 2560, 4096, 9728, 16384):
             try:
                 pl = w4.w4a16_plan(1, N, K, path=w4.PATH_MATVEC_ROWS, sm_count=148)
             except w4.W4A16Error:
                 continue
-            oct_, G = -(-N // 8), K // 128
-            noct = -(-oct_ // pl["grid_x"])
-            assert pl["grid_x"] <= 296 and noct <= 9 and pl["smem_bytes"] == smem(noct, G)
-            if noct < min(-(-oct_ // 148), 9):
-                assert smem(noct + 1, G) > 110 * 1024, (N, K, noct)
+            nh, G, s = -(-N // 8), K // 128, pl["splits"]
+            fits = {}
+            for t in (1, 2, 4):
+                if t > G:
+                    continue
+                cl = min(148 // t, nh)
+                hb = -(-nh // cl)
+                if (hb + 1) // 2 <= 5 and rows_smem(hb, -(-G // t), t) <= 115712:
+                    fits[t] = ((hb + 1) // 2) * (-(-G // t)) // 8
+            enough = [t for t in sorted(fits) if fits[t] >= 4]
+            want = enough[0] if enough else (2 if 2 in fits else min(fits))
+            assert s == want, (N, K, fits, s)
+            assert pl["grid_x"] == (148 // s) * s
+
+
+def test_rows_forced_launch():
+    """row_blocks and splits together fix the launch (tests and sweeps use it)."""
+    pl = w4.w4a16_plan(1, 9728, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148, splits=1, row_blocks=2)
+    assert pl["tiles"] == -(-(9728 // 8) // 4) and pl["row_blocks"] == 2 and pl["splits"] == 1
+    assert pl["grid_x"] == pl["tiles"]   # more clusters than SMs: no padding
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_plan(1, 9728, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148, row_blocks=6)
+    assert e.value.status == w4.ERR_INVALID_ARG
 
 
 @pytest.mark.parametrize("N,K", [(1024, 2560), (4096, 2560), (2560, 4096), (9728, 2560), (2560, 9728),

@@ -89,3 +89,33 @@ def test_back_to_back_static_weights():
     assert w4.w4a16_device_status() == w4.OK
     for p, y in zip(probs, ys):
         assert_close(bits(y), oracle_y(p), "back-to-back")
+
+
+@pytest.mark.parametrize("splits", [1, 2, 3, 4])
+@pytest.mark.parametrize("M,N,K", [(1, 24, 1024), (8, 1000, 768), (5, 2568, 1024), (3, 136, 512)])
+def test_forced_splits_integer_bit_exact(splits, M, N, K):
+    """Every K split of a cluster (uneven group counts for 3), odd half-block counts and
+    clusters padded with CTAs that own no rows: integer problems are exact on every path."""
+    prob = synth.make_integer_problem(M, N, K)
+    d = to_device(prob)
+    y = w4.w4a16_matmul_ex(d["x"], d["wq"], d["scales"], d["biases"], path=w4.PATH_MATVEC_ROWS, splits=splits)
+    torch.cuda.synchronize()
+    assert w4.w4a16_device_status() == w4.OK
+    assert np.array_equal(bits(y), oracle_y(prob)), f"splits={splits} M={M} N={N} K={K}"
+
+
+@pytest.mark.parametrize("splits,row_blocks", [(1, 1), (1, 3), (2, 2), (4, 5), (2, 5)])
+def test_forced_launch_shapes(splits, row_blocks):
+    """Explicit (splits, row blocks) launches of the gate and down projections at M = 8."""
+    for (N, K) in ((9728, 2560), (2560, 9728)):
+        try:
+            w4.w4a16_plan(8, N, K, path=w4.PATH_MATVEC_ROWS, splits=splits, row_blocks=row_blocks)
+        except w4.W4A16Error:
+            continue   # the layout does not fit
+        prob = synth.make_problem(8, N, K)
+        d = to_device(prob)
+        y = w4.w4a16_matmul_ex(d["x"], d["wq"], d["scales"], d["biases"], path=w4.PATH_MATVEC_ROWS,
+                               splits=splits, row_blocks=row_blocks)
+        torch.cuda.synchronize()
+        assert w4.w4a16_device_status() == w4.OK
+        assert_close(bits(y), oracle_y(prob), f"splits={splits} rb={row_blocks} N={N} K={K}")
