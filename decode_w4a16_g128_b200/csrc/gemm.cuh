@@ -7,10 +7,11 @@
 // 32x32x32 Metal tile.
 //
 // Algebra (exact-integer factorisation, per 128-group g):
-//   sum_k x[m,k] w[n,k] = sum_g s[n,g] P'[n,m,g] + sum_g (b[n,g] - 128 s[n,g]) X[m,g],
-//   P'[n,m,g] = sum_{k in g} (128 + q[n,k]) x[m,k],   X[m,g] = sum_{k in g} x[m,k].
-// 128 + q is an exact BF16 value and x is BF16, so every product of P' is
-// exact; only FP32 sums round.
+//   sum_k x[m,k] w[n,k] = sum_g (s[n,g] / 8) P8[n,m,g] + sum_g (b[n,g] - 16 s[n,g]) X[m,g],
+//   P8[n,m,g] = sum_{k in g} (128 + 8 q[n,k]) x[m,k],   X[m,g] = sum_{k in g} x[m,k].
+// 128 + 8 q is an exact BF16 value (the code in mantissa bits 3-6 of 128.0) and x is BF16,
+// so every product of P8 is exact; only FP32 sums round.  The offset 128 is 16 code units,
+// which keeps the cancellation between the two terms small when x is mostly of one sign.
 //
 // Roles of the operands: the tensor cores compute D[n, m] (TMEM lane = weight
 // row n, column = x row m).  The dequantised codes are the A operand and live
@@ -26,7 +27,7 @@
 // X[m,g] as three BF16 pieces whose sum is exactly the FP32 value, twice, and for
 // every weight row n the matching coefficients:
 //   Xs[m, 6g + j] = Xs[m, 6g + 3 + j] = piece j of X[m,g]            (j = 0, 1, 2)
-//   Bc[n, 6g + j] = b[n,g],  Bc[n, 6g + 3 + j] = -128 s[n,g]         (exact BF16)
+//   Bc[n, 6g + j] = b[n,g],  Bc[n, 6g + 3 + j] = -16 s[n,g]          (exact BF16)
 // padded with zeros to Kx = 128 ceil(6 G / 128) columns.  The GEMM runs Kx / 128
 // extra "bias steps" (A = a 128-column block of Bc, B = the same block of Xs),
 // spread round-robin over the K splits and added with scale 1.
@@ -54,6 +55,7 @@
 // launch allocation before the common tail.  All waits are bounded.
 #pragma once
 
+#include "plain.cuh"
 #include "ptx.cuh"
 
 namespace w4a16 {
@@ -126,6 +128,7 @@ __host__ __device__ constexpr int bias_steps(int G) { return (kBiasCoef * G + 12
 __host__ __device__ constexpr int xs_cols(int G) { return 128 * bias_steps(G); }
 
 struct Params {
+    const uint16_t *x;        // bf16 [M, K] (read by TMA; directly only by the plain path)
     const uint32_t *wq;       // [N, G*16] packed codes
     const uint16_t *scales;   // bf16 [N, G]
     const uint16_t *biases;   // bf16 [N, G]
@@ -145,7 +148,7 @@ struct Params {
 // (FP32: each lane of a half-warp sums 8 consecutive values, then the 16 lanes
 // in a fixed tree), X = p0 + p1 + p2 exactly with
 // p0 = bf16(X), p1 = bf16(X - p0), p2 = X - p0 - p1 (exact in BF16).
-// Bc[n, 6g + j] = b[n,g], Bc[n, 6g + 3 + j] = -128 s[n,g] (one thread per (n, g)).
+// Bc[n, 6g + j] = b[n,g], Bc[n, 6g + 3 + j] = -16 s[n,g] (one thread per (n, g)).
 // The last group of a row also writes the zero padding 6G .. Kx-1.
 __global__ void __launch_bounds__(256) prep_kernel(const uint16_t *__restrict__ x, const uint16_t *__restrict__ scales,
                                                    const uint16_t *__restrict__ biases, uint16_t *__restrict__ xs,
@@ -196,7 +199,7 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t *__restrict__ 
         const long long r = item / G;
         const int g = static_cast<int>(item - r * G);
         const uint32_t b = __ldg(biases + r * G + g);
-        const uint32_t t = __bfloat16_as_ushort(__float2bfloat16_rn(-128.f * bf16_to_f32(__ldg(scales + r * G + g))));
+        const uint32_t t = __bfloat16_as_ushort(__float2bfloat16_rn(-16.f * bf16_to_f32(__ldg(scales + r * G + g))));
         uint16_t *row = bc + r * Kx;
         uint32_t *dst = reinterpret_cast<uint32_t *>(row + kBiasCoef * g);
         dst[0] = b | (b << 16);
@@ -209,9 +212,10 @@ __global__ void __launch_bounds__(256) prep_kernel(const uint16_t *__restrict__ 
 
 // ------------------------------------------------------------------ GEMM
 
-__device__ __forceinline__ uint32_t bf16x2_plus128(uint32_t v, uint32_t v4, uint32_t sel) {
-    // bytes sel of (v, v >> 4) -> two codes in bits 0-3 and 16-19 -> BF16 128 + code
-    return codes_to_bf16x2_plus128(prmt(v, v4, sel));
+__device__ __forceinline__ uint32_t bf16x2_128_plus_8q(uint32_t v3, uint32_t v1, uint32_t sel) {
+    // bytes sel of (v3 = v << 3, v1 = v >> 1): byte j of v3 holds code 2j in bits 3-6, byte j
+    // of v1 code 2j + 1 -> two codes in bits 3-6 and 19-22 -> BF16 128 + 8 code
+    return codes_to_bf16x2_128_plus_8q(prmt(v3, v1, sel));
 }
 
 // 64 consecutive 32-bit columns of this thread's lane into registers (warp-collective;
@@ -242,6 +246,15 @@ __device__ __forceinline__ float f32x2_lo(unsigned long long v) { return __uint_
 __device__ __forceinline__ float f32x2_hi(unsigned long long v) { return __uint_as_float(static_cast<uint32_t>(v >> 32)); }
 
 __device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+__device__ __forceinline__ bool bf16_not_finite(uint16_t h) { return (h & 0x7F80u) == 0x7F80u; }
+
+// BF16 of the plain definition of y[m, n] (outputs whose fast result is not finite).
+__device__ __forceinline__ uint16_t plain_output_bf16(const Params &p, long long m, long long n) {
+    const long long G = p.G;
+    return __bfloat16_as_ushort(__float2bfloat16_rn(
+        plain_output(p.x + m * 128 * G, p.wq + n * 16 * G, p.scales + n * G, p.biases + n * G, p.G)));
+}
 
 // Tile t of the output: its x rows start at 128 m, this CTA's weight rows at row0.
 struct TileCoord {
@@ -488,11 +501,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t w[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
                     for (int jj = 0; jj < 8; ++jj) {   // word jj: k = 8 jj .. 8 jj + 7 -> columns 4 jj .. 4 jj + 3
-                        const uint32_t v = w[jj], v4 = v >> 4;
-                        r[4 * jj + 0] = bf16x2_plus128(v, v4, 0x0400u);
-                        r[4 * jj + 1] = bf16x2_plus128(v, v4, 0x0501u);
-                        r[4 * jj + 2] = bf16x2_plus128(v, v4, 0x0602u);
-                        r[4 * jj + 3] = bf16x2_plus128(v, v4, 0x0703u);
+                        const uint32_t v3 = w[jj] << 3, v1 = w[jj] >> 1;
+                        r[4 * jj + 0] = bf16x2_128_plus_8q(v3, v1, 0x0400u);
+                        r[4 * jj + 1] = bf16x2_128_plus_8q(v3, v1, 0x0501u);
+                        r[4 * jj + 2] = bf16x2_128_plus_8q(v3, v1, 0x0602u);
+                        r[4 * jj + 3] = bf16x2_128_plus_8q(v3, v1, 0x0703u);
                     }
                 } else {   // 64 coefficients of this column half (bias steps are few: loaded here)
                     const int t = split + i * p.splits;
@@ -548,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int j = 0; j < 32; ++j) acc2[j] = 0ull;
             for (int i = 0; i < steps && ok; ++i) {
-                const float sc = (row_ok && i >= nbs) ? bf16_to_f32(srow[g0 + i - nbs]) : 1.f;
+                const float sc = (row_ok && i >= nbs) ? 0.125f * bf16_to_f32(srow[g0 + i - nbs]) : 1.f;   // s / 8
                 if (!mbar_wait(&done[ds.slot], ds.phase)) { ok = false; break; }
                 tc_fence_after();
                 uint32_t r[64];
@@ -569,6 +582,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 acc[2 * j] = f32x2_lo(acc2[j]);
                 acc[2 * j + 1] = f32x2_hi(acc2[j]);
             }
+
             __syncwarp();
             if (lane == 0) mbar_arrive(&sc_empty[sb]);   // this tile's scales are no longer read
             if (k == 0) pdl_wait();   // y may still be read by the preceding kernel
@@ -584,9 +598,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // that overlaps the next tile's main loop
                 if (warp == kWarpEpi && lane == 0) bulk_wait_read_all();   // the previous store read it
                 named_bar_sync(kBarEpi, kEpiWarps * 32);
+                unsigned long long bad = 0ull;   // outputs whose fast result is not finite
 #pragma unroll
-                for (int j = 0; j < 64; ++j)
-                    out_tile[(half * 64 + j) * BN + nl] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+                for (int j = 0; j < 64; ++j) {
+                    const uint16_t h = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+                    out_tile[(half * 64 + j) * BN + nl] = h;
+                    if (bf16_not_finite(h)) bad |= 1ull << j;
+                }
+                for (; bad && row_ok; bad &= bad - 1) {   // the plain definition for those (rare)
+                    const int j = __ffsll(static_cast<long long>(bad)) - 1;
+                    if (m0 + j < p.M)
+                        out_tile[(half * 64 + j) * BN + nl] = plain_output_bf16(p, m0 + j, row);
+                }
                 fence_proxy_async_smem();   // the async proxy reads the tile
                 named_bar_sync(kBarEpi, kEpiWarps * 32);
                 if (ok && warp == kWarpEpi && lane == 0) {
@@ -594,10 +617,18 @@ __global__ void __launch_bounds__(kThreads, 1)
                     bulk_commit_group();
                 }
             } else if (row_ok && ok) {
+                unsigned long long bad = 0ull;   // outputs whose fast result is not finite
 #pragma unroll
                 for (int j = 0; j < 64; ++j)
-                    if (m0 + j < p.M)
-                        p.y[static_cast<long long>(m0 + j) * p.N + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+                    if (m0 + j < p.M) {
+                        const uint16_t h = __bfloat16_as_ushort(__float2bfloat16_rn(acc[j]));
+                        p.y[static_cast<long long>(m0 + j) * p.N + row] = h;
+                        if (bf16_not_finite(h)) bad |= 1ull << j;
+                    }
+                for (; bad; bad &= bad - 1) {   // the plain definition for those (rare)
+                    const int j = __ffsll(static_cast<long long>(bad)) - 1;
+                    p.y[static_cast<long long>(m0 + j) * p.N + row] = plain_output_bf16(p, m0 + j, row);
+                }
             }
         }
         if (p.tma_store && warp == kWarpEpi && lane == 0)
@@ -641,6 +672,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const long long mrow = static_cast<long long>(tile_m) * BM + ml;
                 const long long n = row0 + 4 * c4;
                 if (mrow < p.M) {
+                    // outputs whose fast result is not finite: the plain definition
+                    if (!isfinite(v.x) && n < p.N) v.x = plain_output(p.x + mrow * 128ll * G, p.wq + n * 16ll * G, p.scales + n * G, p.biases + n * G, G);
+                    if (!isfinite(v.y) && n + 1 < p.N) v.y = plain_output(p.x + mrow * 128ll * G, p.wq + (n + 1) * 16ll * G, p.scales + (n + 1) * G, p.biases + (n + 1) * G, G);
+                    if (!isfinite(v.z) && n + 2 < p.N) v.z = plain_output(p.x + mrow * 128ll * G, p.wq + (n + 2) * 16ll * G, p.scales + (n + 2) * G, p.biases + (n + 2) * G, G);
+                    if (!isfinite(v.w) && n + 3 < p.N) v.w = plain_output(p.x + mrow * 128ll * G, p.wq + (n + 3) * 16ll * G, p.scales + (n + 3) * G, p.biases + (n + 3) * G, G);
                     uint16_t *dst = p.y + mrow * p.N + n;
                     if (n + 4 <= p.N && (p.N & 3) == 0) {
                         *reinterpret_cast<uint2 *>(dst) = make_uint2(pack_bf16x2(v.x, v.y), pack_bf16x2(v.z, v.w));

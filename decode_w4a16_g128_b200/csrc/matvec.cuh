@@ -44,11 +44,13 @@
 // reduction values):
 //   sum_k x[m,k] w[n,k] = sum_g ( s[n,g] * P[m,n,g] + b[n,g] * X[m,g] ),
 //   P[m,n,g] = sum_{k in g} x[m,k] q[n,k],  X[m,g] = sum_{k in g} x[m,k].
-// Codes enter the MMA as the exact BF16 values 128 + q (one LOP3 per two
-// codes), so the MMA yields P + 128 X; the epilogue applies s and (b - 128 s)
-// once per group in FP32.  Every product is exact; only FP32 sums round.
+// Codes enter the MMA as the exact BF16 values 128 + 8 q (one shift and one
+// LOP3 per two codes), so the MMA yields 8 P + 128 X; the epilogue applies s / 8
+// and (b - 16 s) once per group in FP32.  Every product is exact; only FP32 sums
+// round.
 #pragma once
 
+#include "plain.cuh"
 #include "ptx.cuh"
 
 namespace w4a16 {
@@ -85,6 +87,8 @@ __host__ __device__ constexpr long long smem_bytes(int stages, int slab_slots, l
 }
 
 struct Params {
+    const uint16_t *x;        // bf16 [M, K] (read by TMA; directly only by the plain path)
+    const uint32_t *wq;       // [N, K/8] packed codes (likewise)
     const uint16_t *scales;   // bf16 [N, G]
     const uint16_t *biases;   // bf16 [N, G]
     uint16_t *y;              // bf16 [M, N]
@@ -448,7 +452,7 @@ __global__ void __maxnreg__(80)
             // x sums of group j: prep warps 2 j and 2 j + 1 each summed half of it
             const float2 X0 = lds_f2(xst + 2 * j * (kMaxM * 4));
             const float2 X1 = lds_f2(xst + (2 * j + 1) * (kMaxM * 4));
-            // scale and bias of rows rA, rB for group g; b' = b - 128 s
+            // scale and bias of rows rA, rB for group g; b' = b - 16 s
             uint32_t s0, s1, b0, b1;
             if (slab_rows) {
                 s0 = lds16(sl_s + 2 * (rA * G + g));
@@ -467,17 +471,17 @@ __global__ void __maxnreg__(80)
                 // word r of each row holds codes for 8 consecutive k; fragment r holds the same k
                 const uint32_t w0 = (r == 0) ? wa.x : (r == 1) ? wa.y : (r == 2) ? wa.z : wa.w;
                 const uint32_t w8 = (r == 0) ? wb.x : (r == 1) ? wb.y : (r == 2) ? wb.z : wb.w;
-                const uint32_t a_h0[4] = {codes_to_bf16x2_plus128(w0), codes_to_bf16x2_plus128(w8),
-                                          codes_to_bf16x2_plus128(w0 >> 4), codes_to_bf16x2_plus128(w8 >> 4)};
-                const uint32_t a_h1[4] = {codes_to_bf16x2_plus128(w0 >> 8), codes_to_bf16x2_plus128(w8 >> 8),
-                                          codes_to_bf16x2_plus128(w0 >> 12), codes_to_bf16x2_plus128(w8 >> 12)};
+                const uint32_t a_h0[4] = {codes_to_bf16x2_128_plus_8q(w0 << 3), codes_to_bf16x2_128_plus_8q(w8 << 3),
+                                          codes_to_bf16x2_128_plus_8q(w0 >> 1), codes_to_bf16x2_128_plus_8q(w8 >> 1)};
+                const uint32_t a_h1[4] = {codes_to_bf16x2_128_plus_8q(w0 >> 5), codes_to_bf16x2_128_plus_8q(w8 >> 5),
+                                          codes_to_bf16x2_128_plus_8q(w0 >> 9), codes_to_bf16x2_128_plus_8q(w8 >> 9)};
                 mma_bf16_16816(pacc[0], a_h0, fr[r].x, fr[r].y, pacc[0]);
                 mma_bf16_16816(pacc[1], a_h1, fr[r].z, fr[r].w, pacc[1]);
             }
             // epilogue: rows rA (d0, d1) and rB (d2, d3); x rows 2tq, 2tq+1
             const float Xa = X0.x + X1.x, Xb = X0.y + X1.y;
-            const float sA = bf16_bits_to_f32(s0), sB = bf16_bits_to_f32(s1);
-            const float bA = fmaf(-128.f, sA, bf16_bits_to_f32(b0)), bB = fmaf(-128.f, sB, bf16_bits_to_f32(b1));
+            const float sA = 0.125f * bf16_bits_to_f32(s0), sB = 0.125f * bf16_bits_to_f32(s1);   // s / 8
+            const float bA = fmaf(-128.f, sA, bf16_bits_to_f32(b0)), bB = fmaf(-128.f, sB, bf16_bits_to_f32(b1));   // b - 16 s
             acc[0] = fmaf(bA, Xa, fmaf(sA, pacc[0][0] + pacc[1][0], acc[0]));
             acc[1] = fmaf(bA, Xb, fmaf(sA, pacc[0][1] + pacc[1][1], acc[1]));
             acc[2] = fmaf(bB, Xa, fmaf(sB, pacc[0][2] + pacc[1][2], acc[2]));
@@ -544,6 +548,15 @@ __global__ void __maxnreg__(80)
                 }
             }
         }
+        // outputs whose BF16 result is not finite: the plain definition
+        const long long nn[4] = {nA, nA, nB, nB}, mm[4] = {mA, mB, mA, mB};
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+            if (!isfinite(__bfloat162float(__float2bfloat16_rn(out[e]))) && nn[e] < p.N && mm[e] < p.M) {
+                const long long K = static_cast<long long>(p.G) * 128;
+                out[e] = plain_output(p.x + mm[e] * K, p.wq + nn[e] * (K / 8), p.scales + nn[e] * p.G,
+                                      p.biases + nn[e] * p.G, p.G);
+            }
         if (nA < p.N) {
             if (mA < p.M) p.y[static_cast<long long>(mA) * p.N + nA] = f32_to_bf16_bits(out[0]);
             if (mB < p.M) p.y[static_cast<long long>(mB) * p.N + nA] = f32_to_bf16_bits(out[1]);

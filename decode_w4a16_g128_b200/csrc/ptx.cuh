@@ -233,12 +233,15 @@ __device__ __forceinline__ uint32_t lds32(uint32_t addr) {
 
 // ------------------------------------------------------------------ bit tricks
 
-// Two 4-bit codes -> two BF16 values (128 + code).  Takes bits 0-3 and 16-19
-// of v; the constant 0x4300 is BF16 128.0, whose unit in the last place is 1,
-// so OR-ing a code into the low mantissa bits gives 128 + code exactly.
-__device__ __forceinline__ uint32_t codes_to_bf16x2_plus128(uint32_t v) {
+// Two 4-bit codes -> two BF16 values 128 + 8 code.  Takes bits 3-6 and 19-22 of v: the
+// constant 0x4300 is BF16 128.0, whose seven mantissa bits count units of 1, so OR-ing a
+// code into mantissa bits 3-6 gives 128 + 8 code exactly (the highest position a 4-bit code
+// can take below the exponent).  The offset 128 is then 16 code units, not 128: the group
+// sum of x that removes it again is 8 times smaller, and so is the cancellation between
+// the two terms when x is mostly of one sign.
+__device__ __forceinline__ uint32_t codes_to_bf16x2_128_plus_8q(uint32_t v) {
     uint32_t r;
-    asm("lop3.b32 %0, %1, 0x000F000F, 0x43004300, 0xEA;" : "=r"(r) : "r"(v));
+    asm("lop3.b32 %0, %1, 0x00780078, 0x43004300, 0xEA;" : "=r"(r) : "r"(v));
     return r;
 }
 

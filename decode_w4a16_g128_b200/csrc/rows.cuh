@@ -23,9 +23,9 @@
 // Compute: m16n8k16 BF16 tensor-core MMAs with the CODES as A (16 weight rows
 // x 16 k) and x as B (16 k x 8 columns = the M <= 8 activation rows, zeros
 // beyond M), so every MMA row is a real weight row.  Codes enter as the exact
-// BF16 values 128 + q (one LOP3 per two codes); the MMA yields
-// P' = sum (128 + q) x, and the group sum X = sum x comes from MMAs against
-// all-ones A.  The epilogue adds s P' + (b - 128 s) X in FP32 per group.
+// BF16 values 128 + 8 q (one shift and one LOP3 per two codes); the MMA yields
+// P8 = sum (128 + 8 q) x, and the group sum X = sum x comes from MMAs against
+// all-ones A.  The epilogue adds (s / 8) P8 + (b - 16 s) X in FP32 per group.
 // Lane (g, t) = (lane / 4, lane % 4) reads code words 4t .. 4t+3 of rows g and
 // g + 8 of a row block (k = 32t .. 32t+31 of the group, one 16-byte load per
 // row, conflict-free: a quarter warp covers two 64-byte rows) and the same 32 k
@@ -42,6 +42,7 @@
 // the result does not depend on timing.
 #pragma once
 
+#include "plain.cuh"
 #include "ptx.cuh"
 
 namespace w4a16 {
@@ -85,6 +86,7 @@ __host__ __device__ constexpr long long smem_bytes(int hb, int gc, int s) {
 
 struct Params {
     const uint16_t *x;        // bf16 [M, K]
+    const uint32_t *wq;       // [N, K/8] packed codes (read by TMA; directly only by the plain path)
     const uint16_t *scales;   // bf16 [N, G]
     const uint16_t *biases;   // bf16 [N, G]
     uint16_t *y;              // bf16 [M, N]
@@ -274,22 +276,24 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
                     float da[4] = {0.f, 0.f, 0.f, 0.f}, db[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int c = 0; c < 4; ++c) {
-                        const uint32_t a0[4] = {codes_to_bf16x2_plus128(wa[c]), codes_to_bf16x2_plus128(wb[c]),
-                                                codes_to_bf16x2_plus128(wa[c] >> 4), codes_to_bf16x2_plus128(wb[c] >> 4)};
+                        // nibbles (0,4), (1,5), (2,6), (3,7) moved to bits 3-6 and 19-22
+                        const uint32_t a0[4] = {codes_to_bf16x2_128_plus_8q(wa[c] << 3), codes_to_bf16x2_128_plus_8q(wb[c] << 3),
+                                                codes_to_bf16x2_128_plus_8q(wa[c] >> 1), codes_to_bf16x2_128_plus_8q(wb[c] >> 1)};
                         mma_bf16_16816(da, a0, bf[2 * c][0], bf[2 * c][1], da);
-                        const uint32_t a1[4] = {codes_to_bf16x2_plus128(wa[c] >> 8), codes_to_bf16x2_plus128(wb[c] >> 8),
-                                                codes_to_bf16x2_plus128(wa[c] >> 12), codes_to_bf16x2_plus128(wb[c] >> 12)};
+                        const uint32_t a1[4] = {codes_to_bf16x2_128_plus_8q(wa[c] >> 5), codes_to_bf16x2_128_plus_8q(wb[c] >> 5),
+                                                codes_to_bf16x2_128_plus_8q(wa[c] >> 9), codes_to_bf16x2_128_plus_8q(wb[c] >> 9)};
                         mma_bf16_16816(db, a1, bf[2 * c + 1][0], bf[2 * c + 1][1], db);
                     }
                     // scale and shifted bias of rows 16 rb + g (A row g) and 16 rb + g + 8 (A row g + 8)
                     const int na = (rb * 16 + g) * GCL + gg, nb = na + 8 * GCL;
                     const float sa = bf16_to_f32(sc[na]), sb = bf16_to_f32(sc[nb]);
-                    const float ba = fmaf(-128.f, sa, bf16_to_f32(bi[na]));
-                    const float bb = fmaf(-128.f, sb, bf16_to_f32(bi[nb]));
-                    out[rb][0] = fmaf(ba, X0, fmaf(sa, da[0] + db[0], out[rb][0]));
-                    out[rb][1] = fmaf(ba, X1, fmaf(sa, da[1] + db[1], out[rb][1]));
-                    out[rb][2] = fmaf(bb, X0, fmaf(sb, da[2] + db[2], out[rb][2]));
-                    out[rb][3] = fmaf(bb, X1, fmaf(sb, da[3] + db[3], out[rb][3]));
+                    const float ba = fmaf(-16.f, sa, bf16_to_f32(bi[na]));   // b - 16 s
+                    const float bb = fmaf(-16.f, sb, bf16_to_f32(bi[nb]));
+                    const float s8a = 0.125f * sa, s8b = 0.125f * sb;        // s / 8, exact
+                    out[rb][0] = fmaf(ba, X0, fmaf(s8a, da[0] + db[0], out[rb][0]));
+                    out[rb][1] = fmaf(ba, X1, fmaf(s8a, da[1] + db[1], out[rb][1]));
+                    out[rb][2] = fmaf(bb, X0, fmaf(s8b, da[2] + db[2], out[rb][2]));
+                    out[rb][3] = fmaf(bb, X1, fmaf(s8b, da[3] + db[3], out[rb][3]));
                 }
             }
         }
@@ -314,7 +318,11 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
 #pragma unroll
         for (int ww = 0; ww < kWarps; ++ww) v += src[ww * RB * 16 * kMaxM];
         if (S == 1) {
-            if (r0 + r < p.N) p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            if (r0 + r < p.N) {
+                if (!isfinite(__bfloat162float(__float2bfloat16_rn(v)))) v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8),
+                                                   p.scales + (r0 + r) * G, p.biases + (r0 + r) * G, G);
+                p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
         } else {
             part[r * kMaxM + m] = v;
         }
@@ -336,7 +344,11 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
         const int m = i / RC, r = i - m * RC;
         float v = part[r * kMaxM + m];
         for (int s = 1; s < S; ++s) v += slots[((s - 1) * 16 * RB + r) * kMaxM + m];
-        if (r0 + r < p.N) p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        if (r0 + r < p.N) {
+            if (!isfinite(__bfloat162float(__float2bfloat16_rn(v)))) v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8),
+                                               p.scales + (r0 + r) * G, p.biases + (r0 + r) * G, G);
+            p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        }
     }
 }
 

@@ -517,6 +517,7 @@ int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void
     if (rc) return rc;
     mvr::Params kp;
     kp.x = static_cast<const uint16_t *>(p.x);
+    kp.wq = p.wq;
     kp.scales = static_cast<const uint16_t *>(p.scales);
     kp.biases = static_cast<const uint16_t *>(p.biases);
     kp.y = static_cast<uint16_t *>(p.y);
@@ -578,6 +579,8 @@ int launch_matvec(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_pl
                    static_cast<uint32_t>(p.M), CU_TENSOR_MAP_SWIZZLE_NONE);
     if (rc) return rc;
     mv::Params kp;
+    kp.x = static_cast<const uint16_t *>(p.x);
+    kp.wq = p.wq;
     kp.scales = static_cast<const uint16_t *>(p.scales);
     kp.biases = static_cast<const uint16_t *>(p.biases);
     kp.y = static_cast<uint16_t *>(p.y);
@@ -660,6 +663,7 @@ int launch_gemm(DeviceInfo *d, Workspace *ws, const Problem &p, const w4a16_plan
     }
     // 2. the GEMM (programmatic dependent launch on the group sums)
     gm::Params kp;
+    kp.x = static_cast<const uint16_t *>(p.x);
     kp.wq = p.wq;
     kp.scales = static_cast<const uint16_t *>(p.scales);
     kp.biases = static_cast<const uint16_t *>(p.biases);
@@ -777,8 +781,7 @@ int noalloc_matvec(const Problem &p, void *stream) {
     }
     w4a16_plan_info pl;
     w4a16_options opt = {};
-    opt.path = W4A16_PATH_MATVEC;
-    opt.workers = std::min(d->sms, kNoAllocWorkers);
+    opt.path = W4A16_PATH_MATVEC;   // the stream-K kernel at its measured default CTA count
     plan_matvec(p.M, p.N, p.K, d->sms, &opt, &pl);
     if (pl.tiles > kNoAllocTiles || pl.grid_x > kNoAllocWorkers) return W4A16_ERR_UNSUPPORTED;
     Workspace ws;
@@ -786,7 +789,10 @@ int noalloc_matvec(const Problem &p, void *stream) {
     ws.partial_floats = kNoAllocPartialBytes / sizeof(float);
     ws.tickets = reinterpret_cast<int *>(it->second + kNoAllocPartialBytes);
     ws.ticket_count = kNoAllocTiles;
-    // the flags of this call must start at zero whatever an earlier call left behind
+    // The flags of this call must start at zero whatever an earlier call left behind (a call
+    // that finishes leaves them at zero, one that gave up on a wait may not).  The clearing is
+    // stream-ordered work of its own, so this entry point's kernel never overlaps the end of
+    // the preceding kernel of the stream.
     cudaError_t e = cudaMemsetAsync(ws.tickets, 0, size_t(pl.tiles) * sizeof(int), static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
     return launch_matvec(d, &ws, p, pl, stream, /*pdl=*/true, /*static_weights=*/false);
@@ -869,6 +875,7 @@ int w4a16_device_status(void *stream) {
 
 void w4a16_release(void) {
     std::lock_guard<std::mutex> lock(g_mu);
+    g_noalloc_ptr.clear();   // looked up again on the next call (a device reset may move the array)
     int cur = 0;
     cudaGetDevice(&cur);
     for (auto &kv : g_workspaces) {

@@ -204,9 +204,12 @@ int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u);
  * errors are those of w4a16_matmul.
  * Set-up: the first call on a device looks up the array's device address
  * (cudaGetSymbolAddress); make that first call before any stream capture.
+ * w4a16_release forgets the address; call it before resetting a device.
  * Sharing: every call uses the same array and clears its tickets on `stream`
  * before launching, so calls whose kernels can overlap on the GPU (different
  * streams without ordering) race and give undefined results; serialise them.
+ * That clearing is stream-ordered work of its own: unlike w4a16_matmul, this
+ * entry point's kernel does not overlap the end of the preceding kernel.
  */
 #define W4A16_NOALLOC_MAX_N 1048576
 #define W4A16_NOALLOC_SCRATCH_BYTES 1343488

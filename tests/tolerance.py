@@ -4,14 +4,23 @@ Pass rule: |got - ref| <= ulp_bf16(ref) + 1e-3, with
 ulp_bf16(r) = 2**(floor(log2|r|) - 7) (one unit in the last place of a BF16
 value of that magnitude; 0 for r == 0, leaving the 1e-3 floor).
 
+Infinities match infinities of the same sign; any other non-finite value fails.
+
 The stricter "relative 2**-8 plus 1e-3" reading is half an ulp to one ulp
 depending on where |r| sits in its binade; an honest one-ulp flip between two
 FP32 sums that differ only in their last bits fails it, so it is reported for
 information and not enforced.
 """
+import os
+import sys
+
 import numpy as np
 
 ABS_FLOOR = 1e-3
+
+# (test module, outputs compared, outside the rule, outside the strict form) of every
+# assert_close call, summarised per module at the end of a pytest session
+RECORD = []
 
 
 def bf16_bits_to_f64(bits) -> np.ndarray:
@@ -33,7 +42,9 @@ def compare(got_bits, ref_bits) -> dict:
     if got.shape != ref.shape:
         raise AssertionError(f"shape {got.shape} != {ref.shape}")
     finite = np.isfinite(got) & np.isfinite(ref)
-    d = np.where(finite, np.abs(got - ref), np.inf)
+    same_inf = np.isinf(got) & np.isinf(ref) & (np.sign(got) == np.sign(ref))
+    with np.errstate(invalid="ignore"):   # inf - inf where both are infinite: masked below
+        d = np.where(finite, np.abs(got - ref), np.where(same_inf, 0.0, np.inf))
     tol = ulp_bf16(ref) + ABS_FLOOR
     bad = d > tol
     strict = d > (np.abs(ref) * 2.0 ** -8 + ABS_FLOOR)
@@ -51,5 +62,7 @@ def compare(got_bits, ref_bits) -> dict:
 
 def assert_close(got_bits, ref_bits, what=""):
     r = compare(got_bits, ref_bits)
+    caller = os.path.basename(sys._getframe(1).f_code.co_filename)
+    RECORD.append((caller, r["n"], r["fail"], r["strict_fail"]))
     assert r["fail"] == 0, f"{what}: {r['fail']}/{r['n']} outside 1 ulp + 1e-3 ({r})"
     return r

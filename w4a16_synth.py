@@ -155,3 +155,68 @@ QWEN3_4B_PROJECTIONS = (
     ("down", 9728, 2560),
 )
 QWEN3_4B_LM_HEAD = ("lm_head", 2560, 151936)
+
+
+# ---------------------------------------------------------------- edge-case inputs
+# Inputs built to reach the corners of the layer's definition; none of this computes the
+# layer itself.  Each returns a problem dict like make_problem.
+
+def make_x_positive(rng: np.random.Generator, M: int, K: int, kind: str = "abs4") -> np.ndarray:
+    """Non-zero-mean BF16 activations: ``abs4`` = |N(0,1)| * 4 (mean about 3.2), ``swiglu`` =
+    silu(a) * b with a ~ N(0,1) + 1 and b ~ |N(0,1)| (the mostly positive input of a down
+    projection after the gated activation)."""
+    if kind == "abs4":
+        x = np.abs(rng.standard_normal((M, K), dtype=np.float32)) * np.float32(4)
+    elif kind == "swiglu":
+        a = rng.standard_normal((M, K), dtype=np.float32) + np.float32(1)
+        b = np.abs(rng.standard_normal((M, K), dtype=np.float32))
+        x = (a / (np.float32(1) + np.exp(-a)) * b).astype(np.float32)
+    else:
+        raise ValueError(kind)
+    return bf16_bits(x)
+
+
+def make_edge_problem(M: int, N: int, K: int, x_kind: str = "normal", seed: int = 0) -> dict:
+    """A problem whose weights hit the quantiser's corners and whose activations are chosen
+    by ``x_kind`` (``normal``, ``abs4``, ``swiglu``).
+
+    Weights: W ~ N(0, 0.02), then every 7th (row, group) pair is made constant (the quantiser
+    gives scale 0 and bias = the value, so the group reproduces its bias), and after
+    quantisation every 5th (row, group) pair gets all codes 15 and every 11th all codes 0
+    (scales and biases kept).
+    """
+    rng = shape_rng(M, N, K, seed + 104729)
+    if x_kind == "normal":
+        x = make_x(rng, M, K)
+    else:
+        x = make_x_positive(rng, M, K, x_kind)
+    G = K // GROUP
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    Wg = W.reshape(N, G, GROUP)
+    idx = np.arange(N * G).reshape(N, G)
+    const = (idx % 7) == 3
+    Wg[const] = Wg[const][:, :1]                      # constant group: every value equal
+    wq, s, b = quantize_w4_g128(Wg.reshape(N, K))
+    words = wq.reshape(N, G, GROUP // PACK)
+    words[(idx % 5) == 1] = np.uint32(0xFFFFFFFF)     # all codes 15
+    words[(idx % 11) == 2] = np.uint32(0)             # all codes 0
+    return {"x": x, "wq": words.reshape(N, K // PACK).copy(), "scales": s, "biases": b,
+            "M": M, "N": N, "K": K, "const_groups": int(const.sum())}
+
+
+def make_overflow_problem(M: int, N: int, K: int, sign: float = 1.0, exponent: int = 122,
+                          positive_w: bool = True, seed: int = 0) -> dict:
+    """Huge activations |x| = 2^exponent .. 2^(exponent+1) of one sign.
+
+    With ``positive_w`` (W = 0.05 + |N(0, 0.02)|) every term x * w has the sign of ``sign``,
+    so for exponent 122 the FP32 sum of the plain definition overflows to +-inf for every
+    output.  With W ~ N(0, 0.02) instead, the terms cancel and the plain sums stay finite
+    (about 2^exponent in size) while sums of x alone do not fit FP32 for exponent >= 121."""
+    rng = shape_rng(M, N, K, seed + 15485863)
+    mag = np.float32(2.0 ** exponent) * (np.float32(1) + rng.random((M, K), dtype=np.float32))
+    x = bf16_bits(np.float32(sign) * mag)
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    if positive_w:
+        W = np.float32(0.05) + np.abs(W)
+    wq, s, b = quantize_w4_g128(W)
+    return {"x": x, "wq": wq, "scales": s, "biases": b, "M": M, "N": N, "K": K}
