@@ -35,6 +35,7 @@ PATH_MATVEC_ROWS = 3
 
 FLAG_NO_PDL = 1
 FLAG_STATIC_WEIGHTS = 2
+FLAG_TEST_DROP_COPY = 4
 
 
 class W4A16Error(RuntimeError):

@@ -105,14 +105,15 @@ __device__ __forceinline__ bool status_set() {
 // any thread has recorded a timeout, later waits give up at once (when
 // `give_up_on_status`), so every warp of every CTA leaves its loop quickly.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          bool give_up_on_status = true) {
+                                          bool give_up_on_status = true,
+                                          unsigned long long limit_ns = kWaitTimeoutNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = globaltimer();
     for (uint32_t spin = 1;; ++spin) {
         if (mbar_try_wait_suspend(bar, parity, 20000u)) return true;
         if ((spin & 63u) == 0) {
             if (give_up_on_status && status_set()) return false;
-            if (globaltimer() - t0 > kWaitTimeoutNs) {
+            if (globaltimer() - t0 > limit_ns) {
                 record_timeout();
                 return false;
             }
@@ -537,8 +538,10 @@ __device__ __forceinline__ void st_async_dsmem_f4(uint32_t cluster_addr, float4 
                  : "memory");
 }
 
-// Bounded wait with acquire semantics at cluster scope (for phases completed by remote
-// release arrivals).  Same give-up rules as mbar_wait.
+// Bounded wait with acquire semantics at cluster scope, for phases completed by other CTAs
+// of the cluster (remote release arrivals or st.async bytes).  Unlike mbar_wait it does not
+// give up when another wait has recorded a timeout: the other CTAs always complete the
+// phase, and their stores into this CTA's shared memory must land before this CTA ends.
 __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity) {
     auto test = [&](uint32_t hint) {
         uint32_t ok;
@@ -556,7 +559,6 @@ __device__ __forceinline__ bool mbar_wait_cluster(uint64_t *bar, uint32_t parity
     for (uint32_t spin = 1;; ++spin) {
         if (test(20000u)) return true;
         if ((spin & 63u) == 0) {
-            if (status_set()) return false;
             if (globaltimer() - t0 > kWaitTimeoutNs) {
                 record_timeout();
                 return false;

@@ -40,6 +40,14 @@
 // partials into rank 0's shared memory and arrive on its barrier (release at
 // cluster scope); rank 0 adds them in rank order.  Every sum has a fixed order:
 // the result does not depend on timing.
+//
+// Waits: every wait is on one of this CTA's own copies (rank 0 also waits for its peers'
+// partial sums), bounded by a time limit after which it records W4A16_ERR_TIMEOUT.  Unlike the
+// other kernels' waits they do not give up early when another CTA has recorded a timeout, and
+// a wait that expires does not end the warp's loop: every copy the CTA requested is waited for
+// by the warp that uses it, so none can still be in flight when the CTA's shared memory is
+// reused or released.  A copy that never lands (only the test flag drops one) ends its waits
+// at the limit and leaves the results undefined.
 #pragma once
 
 #include "plain.cuh"
@@ -98,6 +106,8 @@ struct Params {
     int hb_lo, hb_hi;         // floor / ceil(nh / clusters): tm_lo / tm_hi boxes; 8 hb_hi rows per group slot
     int static_weights;       // codes, scales and biases may be read before the dependency wait
     long long x_chunk;        // bytes of x this CTA prefetches into L2 (0: none)
+    int test_drop_copy;       // tests of the timeout path: CTA 0 never loads its first group's codes
+    unsigned long long wait_ns;   // limit of every wait on a copy (kWaitTimeoutNs, shorter in that test)
 };
 
 // BF16 pair (lo, hi) of two words' low / high halves
@@ -161,6 +171,7 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
         prefetch_tmap(tm);
         // codes: box b = words 16 (g0 + b) .. + 15 of rows r0 .. r0 + 8 nhb - 1 (zeros past N)
         for (int b = 0; b < GC; ++b) {
+            if (b == 0 && p.test_drop_copy && blockIdx.x == 0) continue;   // its barrier never completes
             mbar_arrive_expect_tx(&box_full[b], static_cast<uint32_t>(nhb) * 512);
             tma_load_2d(smem + static_cast<long long>(b) * slot, tm, &box_full[b], 16 * (g0 + b),
                         static_cast<int>(r0));
@@ -238,9 +249,9 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
 #pragma unroll
         for (int j = 0; j < kXD; ++j)
             if (ga + j < gb) load_x(xr[j], xrow + (ga + j) * 128, live);
-        bool ok = mbar_wait(sb_full, 0);
+        mbar_wait(sb_full, 0, false, p.wait_ns);
         const uint32_t cbase = smem_u32(smem) + static_cast<uint32_t>(g * 64 + t * 16);
-        for (int gi = ga; ok && gi < gb; gi += kXD) {
+        for (int gi = ga; gi < gb; gi += kXD) {
 #pragma unroll
             for (int j = 0; j < kXD; ++j) {
                 const int gg = gi + j;
@@ -263,7 +274,7 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
                     mma_bf16_16816(xb, ones, bf[2 * c + 1][0], bf[2 * c + 1][1], xb);
                 }
                 const float X0 = xa[0] + xb[0], X1 = xa[1] + xb[1];
-                if (!mbar_wait(&box_full[gg], 0)) { ok = false; break; }
+                mbar_wait(&box_full[gg], 0, false, p.wait_ns);   // after a timeout the results are undefined
                 const int rlo = gg == ga ? u0 - ga * nrb : 0;
                 const int rhi = gg == gb - 1 ? u1 - gg * nrb : nrb;
                 const uint32_t cg = cbase + static_cast<uint32_t>(gg * slot);
@@ -299,7 +310,7 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
         }
     }
     // ---------------------------------------------------------------- fixed-order sums
-    __syncthreads();   // every warp is done with the codes
+    __syncthreads();   // every warp is done with the codes (and every copy of the CTA landed)
     float *red = reinterpret_cast<float *>(smem);   // [warp][row block][row][x row]
 #pragma unroll
     for (int rb = 0; rb < RB; ++rb) {
@@ -319,8 +330,9 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
         for (int ww = 0; ww < kWarps; ++ww) v += src[ww * RB * 16 * kMaxM];
         if (S == 1) {
             if (r0 + r < p.N) {
-                if (!isfinite(__bfloat162float(__float2bfloat16_rn(v)))) v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8),
-                                                   p.scales + (r0 + r) * G, p.biases + (r0 + r) * G, G);
+                if (!isfinite(__bfloat162float(__float2bfloat16_rn(v))))   // not finite: the plain definition
+                    v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8), p.scales + (r0 + r) * G,
+                                     p.biases + (r0 + r) * G, G);
                 p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
             }
         } else {
@@ -339,14 +351,15 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
             st_async_dsmem_f4(dst + 16u * i, reinterpret_cast<const float4 *>(part)[i], bar);
         return;
     }
-    const bool ok = mbar_wait_cluster(red_full, 0);
-    for (int i = tid; ok && i < RM; i += kWarps * 32) {
+    const bool parts = mbar_wait_cluster(red_full, 0);   // the other ranks' partial sums landed
+    for (int i = tid; parts && i < RM; i += kWarps * 32) {
         const int m = i / RC, r = i - m * RC;
         float v = part[r * kMaxM + m];
         for (int s = 1; s < S; ++s) v += slots[((s - 1) * 16 * RB + r) * kMaxM + m];
         if (r0 + r < p.N) {
-            if (!isfinite(__bfloat162float(__float2bfloat16_rn(v)))) v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8),
-                                               p.scales + (r0 + r) * G, p.biases + (r0 + r) * G, G);
+            if (!isfinite(__bfloat162float(__float2bfloat16_rn(v))))   // not finite: the plain definition
+                v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8), p.scales + (r0 + r) * G,
+                                 p.biases + (r0 + r) * G, G);
             p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
         }
     }

@@ -270,7 +270,8 @@ int validate_options(const w4a16_options *opt) {
     if (opt->splits < 0 || opt->splits > gm::kMaxSplits || opt->workers < 0 || opt->sm_count < 0 ||
         opt->row_blocks < 0 || opt->row_blocks > mvr::kMaxRB)
         return W4A16_ERR_INVALID_ARG;
-    if (opt->flags & ~(W4A16_FLAG_NO_PDL | W4A16_FLAG_STATIC_WEIGHTS)) return W4A16_ERR_INVALID_ARG;
+    if (opt->flags & ~(W4A16_FLAG_NO_PDL | W4A16_FLAG_STATIC_WEIGHTS | W4A16_FLAG_TEST_DROP_COPY))
+        return W4A16_ERR_INVALID_ARG;
     return W4A16_OK;
 }
 
@@ -497,7 +498,7 @@ cudaError_t rows_launch_rb(const cudaLaunchConfig_t &cfg, const CUtensorMap &tm_
 }
 
 int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void *stream, bool pdl,
-                bool static_weights) {
+                bool static_weights, bool test_drop_copy) {
     const int G = static_cast<int>(p.K / 128);
     const int rb = pl.row_blocks, S = pl.splits;
     if (rb < 1 || rb > mvr::kMaxRB || S < 1 || S > mvr::kMaxSplits) return W4A16_ERR_INVALID_ARG;
@@ -532,6 +533,8 @@ int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void
     kp.hb_lo = hb_lo;
     kp.hb_hi = hb_hi;
     kp.static_weights = static_weights ? 1 : 0;
+    kp.test_drop_copy = test_drop_copy ? 1 : 0;
+    kp.wait_ns = test_drop_copy ? 200000ull : kWaitTimeoutNs;
     // every CTA prefetches an equal 16-byte-aligned share of x into L2 before the wait
     const long long xbytes = p.M * p.K * 2;
     kp.x_chunk = std::min<long long>(((xbytes + pl.grid_x - 1) / pl.grid_x + 15) / 16 * 16, 65536);
@@ -723,7 +726,9 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     if (rc) return rc;
     const bool pdl = !(opt && (opt->flags & W4A16_FLAG_NO_PDL));
     const bool static_weights = opt && (opt->flags & W4A16_FLAG_STATIC_WEIGHTS);
-    if (pl.path == W4A16_PATH_MATVEC_ROWS) return launch_rows(d, p, pl, stream, pdl, pdl && static_weights);
+    const bool drop = opt && (opt->flags & W4A16_FLAG_TEST_DROP_COPY);
+    if (drop && pl.path != W4A16_PATH_MATVEC_ROWS) return W4A16_ERR_INVALID_ARG;
+    if (pl.path == W4A16_PATH_MATVEC_ROWS) return launch_rows(d, p, pl, stream, pdl, pdl && static_weights, drop);
     if (pl.path == W4A16_PATH_MATVEC) {
         Workspace *ws = nullptr;
         rc = workspace_get(dev, stream, size_t(pl.grid_x) * mv::kPartialFloats, pl.tiles, &ws);

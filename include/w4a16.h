@@ -119,10 +119,18 @@ typedef struct w4a16_options {
  *   not written by work still pending in the stream, so the kernel may start
  *   streaming them before the preceding kernel completes (x is always read
  *   after it).  This is the usual situation for model weights in a decode loop.
+ * W4A16_FLAG_TEST_DROP_COPY: for tests of the timeout path only.  Valid with the
+ *   row-block matvec alone (else W4A16_ERR_INVALID_ARG): CTA 0 never requests the
+ *   codes of its first group, so the waits for them cannot complete, and every
+ *   wait of the launch gives up after 200 us instead of 2 s.  The kernel records
+ *   W4A16_ERR_TIMEOUT (read and cleared by w4a16_device_status), leaves its loops
+ *   and ends normally; the output is undefined.  Nothing traps and the context
+ *   stays usable.
  */
 enum w4a16_flags {
     W4A16_FLAG_NO_PDL = 1,
-    W4A16_FLAG_STATIC_WEIGHTS = 2
+    W4A16_FLAG_STATIC_WEIGHTS = 2,
+    W4A16_FLAG_TEST_DROP_COPY = 4
 };
 
 /*
