@@ -52,7 +52,8 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # the decode step's kernel (the row-block matvec serves all seven projections) and the
 # committed ncu record of its DRAM traffic, valid while these sources are unchanged
 DECODE_KERNEL = "w4a16::mvr::rows_kernel"
-KERNEL_SOURCES = ("decode_w4a16_g128_b200/csrc/rows.cuh", "decode_w4a16_g128_b200/csrc/ptx.cuh")
+KERNEL_SOURCES = ("decode_w4a16_g128_b200/csrc/rows.cuh", "decode_w4a16_g128_b200/csrc/ptx.cuh",
+                  "decode_w4a16_g128_b200/csrc/plain.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rows_decode_traffic.txt")
 
 
