@@ -95,8 +95,12 @@ constexpr int kOffOut = kOffW + kWStages * kWBytes;   // output tile staging for
 constexpr int kOutBytes = BM * BN * 2;                // [x row][weight row] BF16: 32 KB
 constexpr int kOffBar = kOffOut + kOutBytes;
 // Barriers, indexed by step i: ready[i % kXStages] (x or Xs landed + every dequantisation
-// warp stored A), done[i % kXStages] (the step's MMAs completed: frees its x stage, its A
-// buffer and fills its accumulator), d_empty[i % kDBufs] (the epilogue read the accumulator).
+// warp stored A + every epilogue warp read the accumulator of step i - kDBufs, which step i
+// overwrites), done[i % kXStages] (the step's MMAs completed: frees its x stage, its A buffer
+// and fills its accumulator).  The MMA issuer thus waits on one barrier per step: any
+// barrier operation of the issuing thread stalls the tensor pipe for about a hundred cycles
+// (measured: ~110 cycles per step of eight M = 256, N = 128 MMAs for one extra test), so the
+// epilogue's release of an accumulator rides on the ready barrier of the step that reuses it.
 // No waiter can be a whole ring behind the phase it waits for (each role is at most
 // kXStages - 1 steps ahead of the next), so the parities never alias.  Per group j of
 // codes: w_full[j % kWStages] (TMA landed), w_empty[j % kWStages] (dequantisation read it).
@@ -104,7 +108,7 @@ constexpr int kOffBar = kOffOut + kOutBytes;
 // epilogue is done with them), B = scale_bufs(G).  Step, group and tile indices run on
 // across the tiles of a persistent CTA.
 constexpr int kScaleBufsMax = 2;
-constexpr int kNumBars = 2 * kXStages + kDBufs + 2 * kWStages + 2 * kScaleBufsMax;
+constexpr int kNumBars = 2 * kXStages + 2 * kWStages + 2 * kScaleBufsMax;
 static_assert(kABufs < kXStages && kDBufs < kXStages, "one done ring serves every buffer");
 static_assert(kNumBars * 8 + 16 <= 512, "barrier area");
 // The scales of a tile's 128 rows of this CTA, [128][G] BF16, after the barriers: two
@@ -285,8 +289,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
-    uint64_t *ready = bars, *done = ready + kXStages, *d_empty = done + kXStages;
-    uint64_t *w_full = d_empty + kDBufs, *w_empty = w_full + kWStages;
+    uint64_t *ready = bars, *done = ready + kXStages;
+    uint64_t *w_full = done + kXStages, *w_empty = w_full + kWStages;
     uint64_t *sc_full = w_empty + kWStages, *sc_empty = sc_full + kScaleBufsMax;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + kNumBars);
     uint16_t *sc_smem = reinterpret_cast<uint16_t *>(smem + kOffScales);
@@ -322,8 +326,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (threadIdx.x == 0) {
         pdl_launch_dependents();
-        for (int i = 0; i < kXStages; ++i) { mbar_init(&ready[i], 1 + 2 * kDeqWarps); mbar_init(&done[i], 1); }
-        for (int i = 0; i < kDBufs; ++i) mbar_init(&d_empty[i], 2 * kEpiWarps);
+        // ready: the leader's x transaction, the dequantisation and the epilogue warps of both CTAs
+        for (int i = 0; i < kXStages; ++i) { mbar_init(&ready[i], 1 + 2 * kDeqWarps + 2 * kEpiWarps); mbar_init(&done[i], 1); }
         for (int i = 0; i < kWStages; ++i) { mbar_init(&w_full[i], 1); mbar_init(&w_empty[i], kDeqWarps); }
         for (int i = 0; i < kScaleBufsMax; ++i) { mbar_init(&sc_full[i], 1); mbar_init(&sc_empty[i], kEpiWarps); }
         fence_mbar_init();
@@ -338,7 +342,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tmem_base = *tmem_slot;
     // the leader's barriers, as shared::cluster addresses
     const uint32_t ready_l = dsmem_addr(smem_u32(ready), leader);
-    const uint32_t d_empty_l = dsmem_addr(smem_u32(d_empty), leader);
 
     if (warp < kWarpDeq) {
         regs_shrink<kRegsCtl>();
@@ -421,46 +424,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             // -------------------------------------------------------- MMA issuer (pair leader)
             // One thread issues every step: with a second issuing thread on another SM
             // sub-partition, the tensor-memory lanes of both sub-partitions were measured to
-            // receive wrong values now and then.  The tensor pipe takes about one instruction
-            // ahead, so a barrier operation between two steps would leave it idle: while the
-            // last four MMAs of step g run, the thread tests (without blocking) whether step
-            // g+1's inputs are in, and if so starts it with no wait.  The MMAs do not depend
+            // receive wrong values now and then.  Per step it waits on one barrier (the step's
+            // x, A and accumulator are all ready), issues the eight MMAs and one commit, and
+            // nothing else: the tensor pipe holds about one MMA ahead of the issuing thread, and
+            // every further barrier test in the loop would idle it.  The MMAs do not depend
             // on the tile.
             constexpr uint32_t idesc = umma_idesc_bf16(kPairRows, BM);
             const uint16_t mask = static_cast<uint16_t>(3u << leader);
             RingPos<kXStages> xs;      // step g: ready[g % kXStages], its x stage, done[g % kXStages]
             int ab = 0, db = 0;        // A buffer g % kABufs, accumulator g % kDBufs
-            uint32_t dph = 0u;         // bit b: parity of the next d_empty wait of accumulator b
-            bool have = false;         // step g's inputs were seen in the previous step
             for (long long g = 0; g < total; ++g) {
-                if (!have) {
-                    if (!mbar_wait(&ready[xs.slot], xs.phase)) break;
-                    if (g >= kDBufs && !mbar_wait(&d_empty[db], (dph >> db) & 1u)) break;
-                }
-                if (g >= kDBufs) dph ^= 1u << db;
+                if (!mbar_wait_spin(&ready[xs.slot], xs.phase)) break;
                 tc_fence_after();
                 const uint32_t b0 = smem_u32(smem + xs.slot * kXBytes);
                 const uint32_t d = tmem_base + db * BM;
                 const uint32_t a = tmem_base + kACol0 + ab * kACols;
-                RingPos<kXStages> nx = xs;
-                nx.advance();
-                const int ndb = db ^ 1;
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
+                for (int kk = 0; kk < 8; ++kk) {
                     const uint64_t bd = umma_desc_sw128(b0 + (kk >> 2) * kXAtom + (kk & 3) * 32);
                     umma_bf16_ts_pair(d, a + 8 * kk, bd, idesc, kk > 0);
                 }
-                have = g + 1 < total && mbar_test_wait(&ready[nx.slot], nx.phase) &&
-                       (g + 1 < kDBufs || mbar_test_wait(&d_empty[ndb], (dph >> ndb) & 1u));
-#pragma unroll
-                for (int kk = 4; kk < 8; ++kk) {
-                    const uint64_t bd = umma_desc_sw128(b0 + (kk >> 2) * kXAtom + (kk & 3) * 32);
-                    umma_bf16_ts_pair(d, a + 8 * kk, bd, idesc, true);
-                }
                 umma_commit_pair(&done[xs.slot], mask);
-                xs = nx;
+                xs.advance();
                 ab = (ab + 1) & (kABufs - 1);
-                db = ndb;
+                db ^= 1;
             }
         }
         __syncwarp();
@@ -542,8 +529,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nl = quarter * 32 + lane;                         // weight row within the CTA
         const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quarter * 32) << 16) + half * 64;
         RingPos<kXStages> ds;   // step g: done[g % kXStages]
+        RingPos<kXStages> fs;   // step g + kDBufs: ready[...], which the accumulator of step g frees
         int db = 0;
+        long long ge = 0;       // step index across the tiles
         bool ok = true;
+        // the first kDBufs steps find their accumulators free
+        for (int j = 0; j < kDBufs; ++j) {
+            if (lane == 0 && j < total) mbar_arrive_cluster(ready_l + 8 * fs.slot);
+            fs.advance();
+        }
         // Every epilogue warp takes both named barriers of every tile, also after a failed
         // wait, so that none is left waiting on a barrier that the others skipped.
         long long t = tile0;
@@ -569,7 +563,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tmem_ld_wait64(r);
                 tc_fence_before();
                 __syncwarp();
-                if (lane == 0) mbar_arrive_cluster(d_empty_l + 8 * db);
+                if (lane == 0 && ge + kDBufs < total) mbar_arrive_cluster(ready_l + 8 * fs.slot);   // accumulator free
+                fs.advance();
+                ++ge;
                 const unsigned long long sc2 = f32x2(sc, sc);
 #pragma unroll
                 for (int j = 0; j < 32; ++j) ffma2(acc2[j], sc2, r[2 * j], r[2 * j + 1]);

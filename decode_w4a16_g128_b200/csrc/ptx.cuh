@@ -121,6 +121,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
     }
 }
 
+// The same bounded wait without the suspend hint, for a thread whose waits are on the
+// critical path (the MMA issuer): a suspended thread was measured to resume about 60 cycles
+// later than one spinning on try_wait, and the tensor pipe idles meanwhile.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t *bar, uint32_t parity,
+                                               unsigned long long limit_ns = kWaitTimeoutNs) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer();
+    for (uint32_t spin = 1;; ++spin) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((spin & 1023u) == 0) {
+            if (status_set()) return false;
+            if (globaltimer() - t0 > limit_ns) {
+                record_timeout();
+                return false;
+            }
+        }
+    }
+}
+
 // Arrive on an mbarrier given by its shared::cluster address, possibly in another CTA
 // of the cluster (default release semantics at CTA scope: the tcgen05 fences around the
 // barrier order tensor-memory accesses; cluster-scope release would drain the SM's
