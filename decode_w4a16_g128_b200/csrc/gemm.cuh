@@ -126,7 +126,7 @@ constexpr int kWarpCodes = 2;           // TMA producer of the packed codes
 static_assert(kDBufs == 2 && (kABufs & (kABufs - 1)) == 0, "ring arithmetic of the MMA issuer");
 // Split-K partial of a CTA, [BM x rows][BN weight rows] FP32, in the x stages once the loop is over.
 static_assert(BM * BN * 4 <= kXStages * kXBytes, "partial tile must fit in the x stages");
-constexpr int kMaxSplits = 4;           // a cluster holds 2 x splits CTAs: at most 8 (portable size)
+constexpr int kMaxSplits = 8;           // a cluster holds 2 x splits CTAs: up to 16 (non-portable size)
 
 __host__ __device__ constexpr int bias_steps(int G) { return (kBiasCoef * G + 127) / 128; }
 __host__ __device__ constexpr int xs_cols(int G) { return 128 * bias_steps(G); }
@@ -660,11 +660,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int item = t; item < (r_hi - r_lo) * (BN / 4); item += kEpiWarps * 32) {
                 const int ml = r_lo + item / (BN / 4), c4 = item % (BN / 4);
                 const uint32_t off = part0 + (ml * BN + 4 * c4) * 4;
-                float4 v = ld_dsmem_f4(dsmem_addr(off, static_cast<uint32_t>(pair_rank)));
-                for (int sp = 1; sp < S; ++sp) {
-                    const float4 w = ld_dsmem_f4(dsmem_addr(off, static_cast<uint32_t>(2 * sp + pair_rank)));
-                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-                }
+                // every partial in flight at once (a remote load takes about a microsecond),
+                // then added in split order
+                float4 w[kMaxSplits];
+#pragma unroll
+                for (int sp = 0; sp < kMaxSplits; ++sp)
+                    if (sp < S) w[sp] = ld_dsmem_f4(dsmem_addr(off, static_cast<uint32_t>(2 * sp + pair_rank)));
+                float4 v = w[0];
+#pragma unroll
+                for (int sp = 1; sp < kMaxSplits; ++sp)
+                    if (sp < S) {
+                        v.x += w[sp].x; v.y += w[sp].y; v.z += w[sp].z; v.w += w[sp].w;
+                    }
                 const long long mrow = static_cast<long long>(tile_m) * BM + ml;
                 const long long n = row0 + 4 * c4;
                 if (mrow < p.M) {

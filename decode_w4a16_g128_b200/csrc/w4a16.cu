@@ -45,6 +45,7 @@ struct DeviceInfo {
     int sms = 0;
     bool gemm_ok = false;     // the GEMM's register split fits its launch allocation
     int gemm_clusters = 0;    // CTA pairs of the GEMM resident at once (its persistent grid)
+    int gemm_max_splits = 4;  // K splits of the GEMM: 8 where clusters of 16 CTAs can be resident
     PFN_cuTensorMapEncodeTiled_v12000 encode = nullptr;
 };
 
@@ -117,6 +118,8 @@ int device_setup(int dev, DeviceInfo **out) {
             if (e == cudaSuccess)
                 e = cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          gm::smem_bytes(gm::kMaxGroups));
+            if (e == cudaSuccess)   // clusters of 2 x 8 K splits exceed the portable size of 8
+                e = cudaFuncSetAttribute(gm::gemm_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
             if (e != cudaSuccess) return cuda_fail(e);
             // how many CTA pairs of the GEMM the device holds at once: the persistent grid
             // never exceeds it, so that no pair waits for another to finish
@@ -135,6 +138,16 @@ int device_setup(int dev, DeviceInfo **out) {
             e = cudaOccupancyMaxActiveClusters(&clusters, gm::gemm_kernel, &occ);
             if (e != cudaSuccess) return cuda_fail(e);
             d.gemm_clusters = clusters > 0 ? clusters : d.sms / 2;
+            // K splits above 4 take clusters of more than 8 CTAs: only where one fits
+            occ.gridDim = dim3(2 * gm::kMaxSplits, 1, 1);
+            cl.val.clusterDim.x = 2 * gm::kMaxSplits;
+            int big = 0;
+            e = cudaOccupancyMaxActiveClusters(&big, gm::gemm_kernel, &occ);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                big = 0;
+            }
+            d.gemm_max_splits = big > 0 ? gm::kMaxSplits : 4;
         }
         d.ready = true;
     }
@@ -335,9 +348,10 @@ void plan_matvec(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
 
 // Tensor-core GEMM: output tiles of 256 weight rows x 128 x rows, each computed by a
 // CTA pair; K split into `splits` contiguous runs of 128-groups (forced by the
-// options, else chosen to fill the SMs); the splits of a tile form one cluster of
-// 2 x splits CTAs.
-void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, w4a16_plan_info *pl) {
+// options, else chosen to fill the SMs, at most max_splits); the splits of a tile form
+// one cluster of 2 x splits CTAs.
+void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, int max_splits, const w4a16_options *opt,
+               w4a16_plan_info *pl) {
     const int64_t G = K / 128;
     const int64_t tm = (M + gm::BM - 1) / gm::BM, tn = (N + gm::kPairRows - 1) / gm::kPairRows;
     int64_t splits = 1;
@@ -346,10 +360,14 @@ void plan_gemm(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *op
     } else {
         // split K only when the tile pairs leave SMs idle
         const int64_t ctas = 2 * tm * tn;
-        if (ctas < sms) splits = std::min<int64_t>(sms / ctas, gm::kMaxSplits);
+        if (ctas < sms) splits = std::min<int64_t>(sms / ctas, max_splits);
+        // clusters of more than 8 CTAs: only a few fit on the device at once (measured: 10
+        // clusters of 14 and 8 of 16 ran in two waves, slower than the same tiles split in 4),
+        // so more than 4 splits only while the whole grid stays within half of the SMs
+        if (splits > 4 && ctas * splits > sms / 2) splits = 4;
         splits = std::min<int64_t>(splits, G / 2 > 0 ? G / 2 : 1);   // at least two groups per split
     }
-    splits = std::max<int64_t>(1, std::min<int64_t>(std::min<int64_t>(splits, G), gm::kMaxSplits));
+    splits = std::max<int64_t>(1, std::min<int64_t>(splits, G));
     std::memset(pl, 0, sizeof(*pl));
     pl->path = W4A16_PATH_GEMM;
     pl->splits = static_cast<int32_t>(splits);
@@ -446,7 +464,8 @@ void plan_rows(int64_t N, int64_t K, const RowsChoice &c, w4a16_plan_info *pl) {
     pl->workspace_bytes = 0;
 }
 
-int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a16_plan_info *pl) {
+// max_splits: the GEMM's largest K split on this device (forced splits above it are refused)
+int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, int max_splits, w4a16_plan_info *pl) {
     int path = 0;
     int rc = choose_path(M, opt, &path);
     if (rc) return rc;
@@ -468,7 +487,8 @@ int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, w4a
     if ((N + gm::kPairRows - 1) / gm::kPairRows > 65535 || (M + gm::BM - 1) / gm::BM > 65535 ||
         K / 128 > gm::kMaxGroups)
         return W4A16_ERR_UNSUPPORTED;
-    plan_gemm(M, N, K, sms, opt, pl);
+    if (opt && opt->splits > max_splits) return W4A16_ERR_UNSUPPORTED;
+    plan_gemm(M, N, K, sms, max_splits, opt, pl);
     return W4A16_OK;
 }
 
@@ -722,7 +742,7 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
         return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
     }
     w4a16_plan_info pl;
-    rc = plan(p.M, p.N, p.K, opt, d->sms, &pl);
+    rc = plan(p.M, p.N, p.K, opt, d->sms, d->gemm_max_splits, &pl);
     if (rc) return rc;
     const bool pdl = !(opt && (opt->flags & W4A16_FLAG_NO_PDL));
     const bool static_weights = opt && (opt->flags & W4A16_FLAG_STATIC_WEIGHTS);
@@ -853,7 +873,7 @@ int w4a16_plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, w4a16_
         out->path = path;
         return rc;
     }
-    return plan(M, N, K, opt, sms, out);
+    return plan(M, N, K, opt, sms, gm::kMaxSplits, out);
 }
 
 int w4a16_device_status(void *stream) {

@@ -100,8 +100,10 @@ int w4a16_matmul_last_rows(const void *x, const uint32_t *wq, const void *scales
 /* Options for the explicit entry points; zero-initialised means "automatic". */
 typedef struct w4a16_options {
     int32_t path;       /* enum w4a16_path                                                  */
-    int32_t splits;     /* GEMM and row-block matvec: K splits (1..4), each a contiguous run of
-                           128-groups; 0 = auto                                              */
+    int32_t splits;     /* K splits, each a contiguous run of 128-groups; 0 = auto.  GEMM:
+                           1..8 (a cluster of 2 x splits CTAs; above 4 only where the device
+                           holds clusters of 16 CTAs, else W4A16_ERR_UNSUPPORTED); row-block
+                           matvec: 1..4                                                      */
     int32_t workers;    /* stream-K matvec: persistent CTAs sharing the (row-tile x group) units;
                            0 = auto                                                          */
     int32_t sm_count;   /* w4a16_plan only: SM count to plan for; 0 = query the current device */

@@ -90,10 +90,18 @@ def test_bad_options():
     opt = w4.make_options(path=w4.PATH_MATVEC)
     assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
                                P(A + 0x400000), 9, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_UNSUPPORTED
-    for splits in (5, 9):
+    for splits in (9, 17):   # above every path's K-split limit
         opt = w4.make_options(splits=splits)
         assert lib.w4a16_matmul_ex(P(A), P(A + 0x100000), P(A + 0x200000), P(A + 0x300000),
                                    P(A + 0x400000), 2, 8, 256, P(0), ctypes.byref(opt)) == w4.ERR_INVALID_ARG
+
+
+def test_row_block_split_limit():
+    """The row-block matvec splits K over at most 4 CTAs of a cluster (the GEMM over up to 8 pairs)."""
+    for splits in range(5, 9):
+        with pytest.raises(w4.W4A16Error) as e:
+            w4.w4a16_plan(2, 4096, 2560, path=w4.PATH_MATVEC_ROWS, splits=splits, sm_count=148)
+        assert e.value.status == w4.ERR_UNSUPPORTED
 
 
 def test_dispatch_rule():
@@ -207,12 +215,13 @@ def test_streamk_owner_matches_brute_force():
     assert w4.w4a16_streamk_owner(10, 2, 10) == -1
 
 
-@pytest.mark.parametrize("M,N,K,expect_splits", [(128, 4096, 2560, 4), (128, 1024, 2560, 4), (128, 2560, 9728, 4),
+@pytest.mark.parametrize("M,N,K,expect_splits", [(128, 4096, 2560, 4), (128, 1024, 2560, 8), (128, 2560, 9728, 4),
                                                  (128, 9728, 2560, 1), (2048, 4096, 2560, 1), (32, 64, 256, 1),
-                                                 (509, 4096, 9728, 1), (129, 1000, 9728, 4)])
+                                                 (509, 4096, 9728, 1), (129, 1000, 9728, 4), (128, 2560, 4096, 4)])
 def test_gemm_split_plan(M, N, K, expect_splits):
     """Tiles of 256 weight rows x 128 x rows, each on a CTA pair; K is split only while
-    the pairs leave SMs idle, and a tile's splits form one cluster of 2 x splits CTAs.
+    the pairs leave SMs idle (above 4 splits only while the grid stays within half of the
+    SMs), and a tile's splits form one cluster of 2 x splits CTAs.
     Without a split the grid is persistent: one pair per two SMs, looping over the tiles."""
     pl = w4.w4a16_plan(M, N, K, sm_count=148)
     assert pl["path"] == w4.PATH_GEMM
@@ -223,14 +232,14 @@ def test_gemm_split_plan(M, N, K, expect_splits):
         assert (pl["grid_x"], pl["grid_y"], pl["grid_z"]) == (2, min(tiles, 74), 1)
     else:
         assert pl["grid_x"] * pl["grid_y"] * pl["grid_z"] == 2 * tiles * expect_splits
-    assert pl["splits"] <= 4 and pl["splits"] <= K // 128
-    assert pl["cluster"] <= 8
+    assert pl["splits"] <= 8 and pl["splits"] <= K // 128
+    assert pl["cluster"] <= 16
 
 
 def test_gemm_forced_splits_plan():
-    for s in range(1, 5):
+    for s in range(1, 9):
         assert w4.w4a16_plan(300, 1000, 1024, path=w4.PATH_GEMM, splits=s, sm_count=148)["splits"] == s
-    for s in range(5, 9):   # a cluster holds at most 8 CTAs: 4 pairs
+    for s in (9, 16):   # a cluster holds at most 16 CTAs: 8 pairs
         with pytest.raises(w4.W4A16Error):
             w4.w4a16_plan(300, 1000, 1024, path=w4.PATH_GEMM, splits=s, sm_count=148)
     assert w4.w4a16_plan(300, 1000, 256, path=w4.PATH_GEMM, splits=4, sm_count=148)["splits"] == 2   # G = 2

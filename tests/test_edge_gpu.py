@@ -3,7 +3,7 @@ layer's definition.
 
 Each kernel path is forced through w4a16_matmul_ex: the row-block matvec (automatic K split,
 and forced 1 and 2), the stream-K matvec (automatic CTA count, 37 and 148 CTAs) and the
-tensor-core GEMM (K splits 1 to 4).  Inputs:
+tensor-core GEMM (K splits 1 to 4 and 8).  Inputs:
 
 * constant groups (the quantiser gives scale 0, so w = bias), and code blocks forced to all 15
   and all 0, with zero-mean, |N(0,1)| * 4 and silu(a) * b activations, at the 9728-deep down
@@ -41,7 +41,7 @@ MATVEC_PATHS = [
     ("streamk-37", dict(path=w4.PATH_MATVEC, workers=37)),
     ("streamk-148", dict(path=w4.PATH_MATVEC, workers=148)),
 ]
-GEMM_PATHS = [(f"gemm-s{s}", dict(path=w4.PATH_GEMM, splits=s)) for s in (1, 2, 3, 4)]
+GEMM_PATHS = [(f"gemm-s{s}", dict(path=w4.PATH_GEMM, splits=s)) for s in (1, 2, 3, 4, 8)]
 
 
 def run(prob, **kw):

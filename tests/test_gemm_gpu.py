@@ -121,7 +121,7 @@ def test_logits_to_keep_lm_head():
     assert_close(bits(full)[63:64], ref_last, "row 63 of all rows")
 
 
-@pytest.mark.parametrize("splits", [1, 2, 3, 4])
+@pytest.mark.parametrize("splits", [1, 2, 3, 4, 5, 8])
 @pytest.mark.parametrize("M,N,K", [(128, 1000, 1024), (300, 257, 1024), (17, 130, 768), (64, 100, 1024)])
 def test_split_k_integer_bit_exact(splits, M, N, K):
     prob = synth.make_integer_problem(M, N, K)
@@ -129,7 +129,7 @@ def test_split_k_integer_bit_exact(splits, M, N, K):
     assert np.array_equal(got, oracle_y(prob)), f"splits={splits} M={M} N={N} K={K}"
 
 
-@pytest.mark.parametrize("splits", [2, 3, 4])
+@pytest.mark.parametrize("splits", [2, 3, 4, 6, 8])
 def test_split_k_down_proj(splits):
     prob = synth.make_problem(128, 2560, 9728, outliers=True)
     assert_close(run(prob, path=w4.PATH_GEMM, splits=splits), oracle_y(prob), f"down_proj splits={splits}")
