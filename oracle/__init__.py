@@ -26,11 +26,12 @@ SOURCE = os.path.join(HERE, "w4a16_oracle.c")
 LIBRARY = os.path.join(HERE, "libw4a16_oracle.so")
 CFLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
           "-std=c11", "-Wall", "-Wextra", "-Werror"]
+LIBS = ["-lm"]
 
 
 def compile_source(src: str, out: str) -> str:
     tmp = out + f".tmp{os.getpid()}"
-    subprocess.run(["gcc", *CFLAGS, src, "-o", tmp], check=True)
+    subprocess.run(["gcc", *CFLAGS, src, "-o", tmp, *LIBS], check=True)
     os.replace(tmp, out)
     return out
 
@@ -66,6 +67,10 @@ class Oracle:
         lib.w4a16_oracle_threads.restype = ctypes.c_int
         lib.w4a16_oracle_set_threads.argtypes = [ctypes.c_int]
         lib.w4a16_oracle_set_threads.restype = None
+        for name in ("w4a16_oracle_quantize", "w4a16_oracle_quantize_bf16"):
+            fn = getattr(lib, name)
+            fn.argtypes = [p, p, p, p, i64, i64]
+            fn.restype = ctypes.c_int
         self.lib = lib
         self.path = path
 
@@ -112,6 +117,26 @@ class Oracle:
         self.lib.w4a16_oracle_round_bf16(pa, out.ctypes.data_as(ctypes.c_void_p), a.size)
         return out
 
+    def quantize(self, w):
+        """W [N,K] (float32 values, or uint16 BF16 bit patterns) -> (wq uint32 [N,K/8],
+        scales uint16 [N,K/128], biases uint16 [N,K/128]) by the min/max recipe."""
+        w = np.asarray(w)
+        if w.ndim != 2:
+            raise ValueError("W must be [N, K]")
+        if w.dtype == np.uint16:
+            fn, w = self.lib.w4a16_oracle_quantize_bf16, np.ascontiguousarray(w)
+        else:
+            fn, w = self.lib.w4a16_oracle_quantize, np.ascontiguousarray(w, dtype=np.float32)
+        N, K = w.shape
+        G = K // 128 if K % 128 == 0 else 0
+        wq = np.empty((N, K // 8), dtype=np.uint32)
+        s = np.empty((N, G), dtype=np.uint16)
+        b = np.empty((N, G), dtype=np.uint16)
+        vp = ctypes.c_void_p
+        if fn(w.ctypes.data_as(vp), wq.ctypes.data_as(vp), s.ctypes.data_as(vp), b.ctypes.data_as(vp), N, K):
+            raise ValueError("oracle rejected its arguments")
+        return wq, s, b
+
     def threads(self) -> int:
         return self.lib.w4a16_oracle_threads()
 
@@ -145,6 +170,10 @@ def unpack(wq, K):
 
 def round_bf16(a):
     return default().round_bf16(a)
+
+
+def quantize(w):
+    return default().quantize(w)
 
 
 def threads():

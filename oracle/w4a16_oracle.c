@@ -22,8 +22,15 @@
  * Outputs are independent, so they may be computed by several threads; the
  * arithmetic of each output is the sequence above regardless.
  *
+ * The quantiser (w4a16_oracle_quantize) produces the packed format above from
+ * FP32 or BF16 weights.  Its recipe is the one the reference problem's inputs
+ * are made with (affine min/max quantisation per 128-group: scale = (max - min)
+ * / 15, bias = min, q = round and clamp to 0..15, eight codes per uint32 low
+ * nibble first); the steps are spelled out above the function.
+ *
  * BF16 values are passed as uint16_t bit patterns.
  */
+#include <math.h>
 #include <stdint.h>
 #include <string.h>
 #ifdef _OPENMP
@@ -156,4 +163,87 @@ void w4a16_oracle_set_threads(int n)
 #else
     (void)n;
 #endif
+}
+
+/*
+ * Quantiser, one 128-group v[0..127] of one weight row:
+ *   1. lo = min, hi = max of the 128 values (compared in k order); a zero lo or hi
+ *      is taken as +0, so the result does not depend on the order of the values
+ *   2. scale = bf16_rne((hi - lo) / 15)    FP32 subtraction, FP32 division
+ *      bias  = bf16_rne(lo)
+ *   3. with sc, bi the BF16 scale and bias widened to FP32:
+ *      q[k] = 0 when sc == 0 (a constant group), else
+ *      q[k] = clamp(nearbyint((v[k] - bi) / sc), 0, 15)   FP32 subtraction and
+ *             division, nearbyint in the default rounding mode (half to even)
+ *   4. word j of the group = sum over i < 8 of q[8 j + i] << (4 i)
+ * Inputs must be finite.
+ */
+static void quantize_group(const float *v, uint32_t *words, uint16_t *scale, uint16_t *bias)
+{
+    float lo = v[0], hi = v[0];
+    for (int j = 1; j < 128; ++j) {
+        if (v[j] < lo)
+            lo = v[j];
+        if (v[j] > hi)
+            hi = v[j];
+    }
+    if (lo == 0.0f)
+        lo = 0.0f;
+    if (hi == 0.0f)
+        hi = 0.0f;
+    const float range = hi - lo;
+    const float step = range / 15.0f;
+    *scale = f32_to_bf16_rne(step);
+    *bias = f32_to_bf16_rne(lo);
+    const float sc = bf16_to_f32(*scale);
+    const float bi = bf16_to_f32(*bias);
+    for (int j = 0; j < 16; ++j)
+        words[j] = 0u;
+    for (int j = 0; j < 128; ++j) {
+        uint32_t code = 0u;
+        if (sc != 0.0f) {
+            const float d = v[j] - bi;
+            const float t = d / sc;
+            const float r = nearbyintf(t);
+            code = r < 0.0f ? 0u : (r > 15.0f ? 15u : (uint32_t)r);
+        }
+        words[j / 8] |= code << (4 * (j % 8));
+    }
+}
+
+static int quantize_check(const void *w, const void *wq, const void *s, const void *b, int64_t N, int64_t K)
+{
+    if (N < 0 || K < 0 || K % 128 != 0)
+        return 1;
+    if (N > 0 && K > 0 && (!w || !wq || !s || !b))
+        return 1;
+    return 0;
+}
+
+/* W [N,K] FP32 -> wq [N,K/8], scales and biases [N,K/128] BF16 bits. */
+int w4a16_oracle_quantize(const float *w, uint32_t *wq, uint16_t *s, uint16_t *b, int64_t N, int64_t K)
+{
+    if (quantize_check(w, wq, s, b, N, K))
+        return 1;
+    const int64_t G = K / 128;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g)
+            quantize_group(w + n * K + g * 128, wq + n * (K / 8) + g * 16, s + n * G + g, b + n * G + g);
+    return 0;
+}
+
+/* The same from BF16 weights: each value widened to FP32 (exactly), then as above. */
+int w4a16_oracle_quantize_bf16(const uint16_t *w, uint32_t *wq, uint16_t *s, uint16_t *b, int64_t N, int64_t K)
+{
+    if (quantize_check(w, wq, s, b, N, K))
+        return 1;
+    const int64_t G = K / 128;
+    float v[128];
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g) {
+            for (int j = 0; j < 128; ++j)
+                v[j] = bf16_to_f32(w[n * K + g * 128 + j]);
+            quantize_group(v, wq + n * (K / 8) + g * 16, s + n * G + g, b + n * G + g);
+        }
+    return 0;
 }

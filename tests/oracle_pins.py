@@ -235,6 +235,95 @@ def pin_rejects_bad_k(orc):
     raise AssertionError("K % 128 != 0 was accepted")
 
 
+# ------------------------------------------------------------------ quantiser pins
+# The recipe of the reference problem's inputs (affine min/max per 128-group: scale =
+# (max - min) / 15 and bias = min, both rounded to BF16 first, q = rint((w - bias) /
+# scale) clamped to 0..15, packed low nibble first).
+
+def _pack_codes(codes):
+    """The packed format's words for a list of codes (eight per word, low nibble first)."""
+    words = []
+    for j in range(0, len(codes), 8):
+        w = 0
+        for i, c in enumerate(codes[j:j + 8]):
+            w |= int(c) << (4 * i)
+        words.append(w)
+    return words
+
+
+def pin_quantize_hand_group(orc):
+    """v_k = 1 + (k % 16) / 8: min 1, max 2.875, step 1.875 / 15 = 0.125 exactly, so the
+    scale is 0.125 (0x3E00), the bias 1.0 (0x3F80) and code k is k % 16."""
+    v = np.array([1.0 + (k % 16) / 8.0 for k in range(128)], np.float32)
+    expect_words = [0x76543210, 0xFEDCBA98] * 8
+    for w in (v[None, :], synth.bf16_bits(v)[None, :]):     # FP32 and BF16 inputs (exact in both)
+        wq, s, b = orc.quantize(w)
+        assert int(s[0, 0]) == 0x3E00 and int(b[0, 0]) == 0x3F80, (hex(s[0, 0]), hex(b[0, 0]))
+        assert [int(x) for x in wq[0]] == expect_words, [hex(int(x)) for x in wq[0]]
+
+
+def pin_quantize_constant_group(orc):
+    """A constant group: scale 0, bias = the value rounded to BF16, every code 0.  0.3 in
+    FP32 is 0x3E99999A; its BF16 rounding is 0x3E9A (the dropped half 0x999A > 0x8000)."""
+    wq, s, b = orc.quantize(np.full((1, 256), 0.3, np.float32))
+    assert s.tolist() == [[0, 0]] and b.tolist() == [[0x3E9A, 0x3E9A]]
+    assert not wq.any()
+
+
+def pin_quantize_ties_to_even(orc):
+    """min 0, max 15: scale 1, bias 0, and a code is the value rounded half to even."""
+    v = np.full(128, 5.0, np.float32)
+    vals = [0.0, 15.0, 2.5, 3.5, 14.5, 0.5, 1.5, 7.49, 12.5, 9.51]
+    codes = [0, 15, 2, 4, 14, 0, 2, 7, 12, 10]
+    v[:len(vals)] = vals
+    wq, s, b = orc.quantize(v[None, :])
+    assert int(s[0, 0]) == 0x3F80 and int(b[0, 0]) == 0
+    expect = codes + [5] * (128 - len(codes))
+    assert [int(x) for x in wq[0]] == _pack_codes(expect), [hex(int(x)) for x in wq[0]]
+
+
+def pin_quantize_signed_zero(orc):
+    """A zero minimum or maximum is taken as +0 whatever the order of -0 and +0."""
+    v = np.linspace(0.0, 1.5, 128).astype(np.float32)
+    a = v.copy(); a[0] = -0.0; a[1] = 0.0      # -0 first
+    c = v.copy(); c[0] = 0.0; c[1] = -0.0      # +0 first
+    d = -v[::-1].copy(); d[-1] = -0.0          # maximum -0
+    wq, s, b = orc.quantize(np.stack([a, c]))
+    assert b.tolist() == [[0], [0]], b
+    assert np.array_equal(wq[0], wq[1]) and s[0, 0] == s[1, 0]
+    d2 = d.copy(); d2[-1] = 0.0                # the same group with +0 as its maximum
+    for x, y in zip(orc.quantize(d[None, :]), orc.quantize(d2[None, :])):
+        assert np.array_equal(x, y)
+
+
+def pin_quantize_matches_numpy_recipe(orc):
+    """The recipe restated with numpy's IEEE float32 operations (w4a16_synth, an independent
+    implementation) on N(0, 0.02) rows and on groups built to reach the clamps: values far
+    from zero with a narrow range, so that the BF16 bias lies well away from the minimum
+    ((w - bias) / scale outside 0..15 before the clamp), and steps that round up or down."""
+    rng = np.random.default_rng([2024, 11])
+    W = rng.standard_normal((48, 512)).astype(np.float32) * np.float32(0.02)
+    off = np.float32(100.2) + rng.random((8, 128), dtype=np.float32)      # lo near 100.2, range < 1
+    W[:8, :128] = off
+    W[8:16, 128:256] = np.float32(-37.7) + np.float32(0.25) * rng.random((8, 128), dtype=np.float32)
+    W[16:24, 256:384] = np.float32(3.0e-3) * rng.standard_normal((8, 128), dtype=np.float32) + np.float32(0.7)
+    got = orc.quantize(W)
+    ref = synth.quantize_w4_g128(W)
+    for g, r, name in zip(got, ref, ("wq", "scales", "biases")):
+        assert np.array_equal(g, r), name
+    # the clamps were reached: some codes 0 and 15 in the offset groups
+    q = (ref[0][:8, :16, None] >> (4 * np.arange(8, dtype=np.uint32))) & 15
+    assert (q == 15).any() and (q == 0).any()
+
+
+def pin_quantize_rejects_bad_k(orc):
+    try:
+        orc.quantize(np.zeros((1, 136), np.float32))
+    except ValueError:
+        return
+    raise AssertionError("K % 128 != 0 was accepted")
+
+
 ALL_PINS = (
     pin_unpack_hand_words,
     pin_onehot_reads_codes,
@@ -246,6 +335,12 @@ ALL_PINS = (
     pin_matmul_golden_cases,
     pin_rational_brute_force,
     pin_rejects_bad_k,
+    pin_quantize_hand_group,
+    pin_quantize_constant_group,
+    pin_quantize_ties_to_even,
+    pin_quantize_signed_zero,
+    pin_quantize_matches_numpy_recipe,
+    pin_quantize_rejects_bad_k,
 )
 
 

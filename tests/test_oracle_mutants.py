@@ -30,6 +30,16 @@ MUTANTS = {
     "truncating_round": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0u;"),
     "ties_away": ("u += 0x7fffu + ((u >> 16) & 1u);", "u += 0x8000u;"),
     "k_descending": ("for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = K - 1; k >= 0; --k) {"),
+    # quantiser
+    "quant_truncates": ("const float r = nearbyintf(t);", "const float r = truncf(t);"),
+    "quant_ties_away": ("const float r = nearbyintf(t);", "const float r = roundf(t);"),
+    "quant_step_16": ("const float step = range / 15.0f;", "const float step = range / 16.0f;"),
+    "quant_bias_unrounded": ("const float bi = bf16_to_f32(*bias);", "const float bi = lo;"),
+    "quant_no_upper_clamp": ("(r > 15.0f ? 15u : (uint32_t)r)", "((uint32_t)r & 0xFu)"),
+    "quant_min_as_max": ("if (v[j] < lo)", "if (v[j] > lo)"),
+    "quant_zero_sign_kept": ("    if (lo == 0.0f)\n        lo = 0.0f;\n", ""),
+    "quant_words_not_cleared": ("        words[j] = 0u;", "        words[j] = 1u;"),
+    "quant_nibble_order": ("code << (4 * (j % 8))", "code << (4 * (7 - j % 8))"),
 }
 
 
@@ -38,7 +48,7 @@ def _build(tmp_path, name, src_text, extra_flags=()):
     src.write_text(src_text)
     out = tmp_path / f"lib{name}.so"
     flags = [f for f in oracle.CFLAGS if f != "-Werror"]   # a mutant may leave a variable unused
-    subprocess.run(["gcc", *flags, *extra_flags, str(src), "-o", str(out)], check=True)
+    subprocess.run(["gcc", *flags, *extra_flags, str(src), "-o", str(out), *oracle.LIBS], check=True)
     return str(out)
 
 
