@@ -67,6 +67,8 @@ class Oracle:
         lib.w4a16_oracle_threads.restype = ctypes.c_int
         lib.w4a16_oracle_set_threads.argtypes = [ctypes.c_int]
         lib.w4a16_oracle_set_threads.restype = None
+        lib.w4a16_oracle_gate_up.argtypes = [p, p, p, p, p, i64, i64, i64]
+        lib.w4a16_oracle_gate_up.restype = ctypes.c_int
         for name in ("w4a16_oracle_quantize", "w4a16_oracle_quantize_bf16"):
             fn = getattr(lib, name)
             fn.argtypes = [p, p, p, p, i64, i64]
@@ -102,6 +104,16 @@ class Oracle:
         if self.lib.w4a16_oracle_matmul_f32(*ptrs, acc.ctypes.data_as(ctypes.c_void_p), M, N, K):
             raise ValueError("oracle rejected its arguments")
         return acc
+
+    def gate_up(self, x, wq, scales, biases) -> np.ndarray:
+        """h [M, N2] BF16 bits = silu(gate) * up over interleaved gate/up rows (2 N2 rows)."""
+        keep, ptrs, M, N, K = self._inputs(x, wq, scales, biases)
+        if N % 16:
+            raise ValueError("gate/up rows come in blocks of 16")
+        h = np.empty((M, N // 2), dtype=np.uint16)
+        if self.lib.w4a16_oracle_gate_up(*ptrs, h.ctypes.data_as(ctypes.c_void_p), M, N // 2, K):
+            raise ValueError("oracle rejected its arguments")
+        return h
 
     def unpack(self, wq, K: int) -> np.ndarray:
         wq, pw = _c(wq, np.uint32)
@@ -162,6 +174,20 @@ def matmul(x, wq, scales, biases):
 
 def matmul_f32(x, wq, scales, biases):
     return default().matmul_f32(x, wq, scales, biases)
+
+
+def gate_up(x, wq, scales, biases):
+    return default().gate_up(x, wq, scales, biases)
+
+
+def interleave_gate_up(gate, up):
+    """Row-interleave two [N2, ...] arrays (a packed layer's wq, scales or biases) in blocks
+    of 8: gate rows 8 b .. 8 b + 7, then up rows 8 b .. 8 b + 7 (a layout, no arithmetic)."""
+    gate, up = np.asarray(gate), np.asarray(up)
+    if gate.shape != up.shape or gate.shape[0] % 8:
+        raise ValueError("gate and up need the same shape and a row count divisible by 8")
+    n2 = gate.shape[0]
+    return np.stack([gate.reshape(n2 // 8, 8, -1), up.reshape(n2 // 8, 8, -1)], axis=1).reshape(2 * n2, -1)
 
 
 def unpack(wq, K):

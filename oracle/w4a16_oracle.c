@@ -126,6 +126,36 @@ int w4a16_oracle_matmul_f32(const uint16_t *x, const uint32_t *wq, const uint16_
     return 0;
 }
 
+/*
+ * Fused gate/up projection with the SwiGLU product.  wq, s, b hold 2 N2 rows, the
+ * gate and up layers interleaved in blocks of 8: rows 16 (j / 8) + j % 8 (gate j) and
+ * 16 (j / 8) + 8 + j % 8 (up j).  For each output:
+ *   g, u = the plain dots of the gate and up rows (steps 1-3 above, FP32)
+ *   h    = bf16_rne((float)(silu(g) * u)), silu(g) = g / (1 + exp(-g)) in double
+ * (the product is rounded to FP32, then to BF16).
+ */
+static double silu(double g)
+{
+    return g / (1.0 + exp(-g));
+}
+
+int w4a16_oracle_gate_up(const uint16_t *x, const uint32_t *wq, const uint16_t *s,
+                         const uint16_t *b, uint16_t *h, int64_t M, int64_t N2, int64_t K)
+{
+    if (N2 < 0 || N2 % 8 != 0 || check(x, wq, s, b, h, M, 2 * N2, K))
+        return 1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t j = 0; j < N2; ++j) {
+            const int64_t gate_row = 16 * (j / 8) + j % 8;
+            const int64_t up_row = gate_row + 8;
+            const double gv = (double)dot_fp32(x, wq, s, b, K, m, gate_row);
+            const double uv = (double)dot_fp32(x, wq, s, b, K, m, up_row);
+            h[m * N2 + j] = f32_to_bf16_rne((float)(silu(gv) * uv));
+        }
+    return 0;
+}
+
 /* Step 1 alone: q[N,K] codes as bytes. */
 int w4a16_oracle_unpack(const uint32_t *wq, uint8_t *q, int64_t N, int64_t K)
 {

@@ -324,6 +324,72 @@ def pin_quantize_rejects_bad_k(orc):
     raise AssertionError("K % 128 != 0 was accepted")
 
 
+# ------------------------------------------------------------------ fused gate/up pins
+# h = bf16(silu(g) * u) over gate/up rows interleaved in blocks of 8.
+
+def _gate_up_problem(gvals, uvals, K=128):
+    """One x row of ones [1, K] and per output a gate row and an up row whose dot with x
+    is the given integer: codes q and scale 1, so the sum is sum(q) + K * bias (exact)."""
+    n2 = len(gvals)
+    assert n2 % 8 == 0
+    def rows(vals):
+        q = np.zeros((n2, K), np.uint8)
+        bias = np.zeros((n2, K // 128), np.float32)
+        for j, v in enumerate(vals):
+            base = int(np.floor(v / K))            # bias per element, the rest from the codes
+            rest = int(v - base * K)
+            assert 0 <= rest <= 15 * K
+            q[j, :rest // 15] = 15
+            q[j, rest // 15] = rest % 15 if rest // 15 < K else 0
+            bias[j, :] = base
+        return synth.pack_nibbles(q), synth.bf16_bits(np.ones((n2, K // 128), np.float32)), synth.bf16_bits(bias)
+    gq, gs, gb = rows(gvals)
+    uq, us, ub = rows(uvals)
+    from oracle import interleave_gate_up
+    x = synth.bf16_bits(np.ones((1, K), np.float32))
+    return x, interleave_gate_up(gq, uq), interleave_gate_up(gs, us), interleave_gate_up(gb, ub)
+
+
+def pin_gate_up_closed_forms(orc):
+    """silu(0) = 0, so g = 0 gives +0 for any u; u = 0 gives +0 (g >= 0); for g >= 64,
+    exp(-g) < 2^-92 and silu(g) = g in double, so h = bf16(g * u) exactly; for g <= -256,
+    silu(g) * u is below the smallest BF16 subnormal and h is a zero of u's sign times g's."""
+    g = [0, 0, 64, 100, 700, -256, -300, 5, 0, 64, 1000, 100, -1000, 3, 0, 0]
+    u = [7, -3, 2, -5, 1, 9, -4, 0, 0, 1, 3, 100, 1, 0, 1, 1000]
+    x, wq, s, b = _gate_up_problem(g, u)
+    h = orc.gate_up(x, wq, s, b)[0]
+    want = {0: 0x0000, 1: 0x8000, 7: 0x0000, 8: 0x0000, 13: 0x0000, 14: 0x0000, 15: 0x0000}
+    for j, bits in want.items():
+        assert int(h[j]) in (bits, bits ^ 0x8000) and _bits_to_fraction(int(h[j])) == 0, (j, hex(h[j]))
+    for j in (2, 3, 4, 9, 10, 11):
+        assert int(h[j]) == int(synth.bf16_bits(np.array([g[j] * u[j]], np.float32))[0]), (j, hex(h[j]))
+    for j in (5, 6, 12):
+        assert _bits_to_fraction(int(h[j])) == 0, (j, hex(h[j]))
+
+
+def pin_gate_up_interleave(orc):
+    """The fused op reads gate j from row 16 (j / 8) + j % 8 and up j eight rows later: with
+    u = 1 and g >= 64 on every output, h is the gate layer's own output, column by column."""
+    rng = np.random.default_rng([77, 1])
+    g = [int(v) for v in rng.integers(64, 1900, 24)]
+    x, wq, s, b = _gate_up_problem(g, [1] * 24)
+    h = orc.gate_up(x, wq, s, b)[0]
+    assert [int(v) for v in h] == [int(v) for v in synth.bf16_bits(np.array(g, np.float32))]
+
+
+def pin_gate_up_odd_part(orc):
+    """silu(g) - silu(-g) = g: for u = 1 the outputs of g and -g differ by g up to the two
+    BF16 roundings (half an ulp of each output)."""
+    gs = [1, 2, 3, 5, 8, 13, 21, 34]
+    g = gs + [-v for v in gs]
+    x, wq, s, b = _gate_up_problem(g, [1] * 16)
+    h = orc.gate_up(x, wq, s, b)[0]
+    for j, v in enumerate(gs):
+        hp, hn = _bits_to_fraction(int(h[j])), _bits_to_fraction(int(h[j + 8]))
+        tol = (abs(hp) + abs(hn)) / 256 + Fraction(1, 1 << 20)
+        assert abs(hp - hn - v) <= tol, (v, float(hp), float(hn))
+
+
 ALL_PINS = (
     pin_unpack_hand_words,
     pin_onehot_reads_codes,
@@ -341,6 +407,9 @@ ALL_PINS = (
     pin_quantize_signed_zero,
     pin_quantize_matches_numpy_recipe,
     pin_quantize_rejects_bad_k,
+    pin_gate_up_closed_forms,
+    pin_gate_up_interleave,
+    pin_gate_up_odd_part,
 )
 
 

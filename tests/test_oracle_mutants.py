@@ -40,6 +40,11 @@ MUTANTS = {
     "quant_zero_sign_kept": ("    if (lo == 0.0f)\n        lo = 0.0f;\n", ""),
     "quant_words_not_cleared": ("        words[j] = 0u;", "        words[j] = 1u;"),
     "quant_nibble_order": ("code << (4 * (j % 8))", "code << (4 * (7 - j % 8))"),
+    # fused gate/up
+    "gate_rows_not_interleaved": ("gate_row = 16 * (j / 8) + j % 8;", "gate_row = 8 * (j / 8) + j % 8;"),
+    "up_row_is_gate_row": ("const int64_t up_row = gate_row + 8;", "const int64_t up_row = gate_row;"),
+    "silu_sign": ("return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
+    "silu_dropped": ("f32_to_bf16_rne((float)(silu(gv) * uv))", "f32_to_bf16_rne((float)(gv * uv))"),
 }
 
 
