@@ -433,9 +433,22 @@ def run_ours(args, world, rank, local):
         while t < args.cpu_seconds or reps == 0:   # whole decode steps until the time bound is reached
             b_, t_ = cpu_sample(weights, xs, 1.0)
             nb, t, reps = nb + b_, t + t_, reps + 1
-        cpu = {"value": round(nb / t / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+        cores = oracle.threads()
+        cpu = {"value": round(nb / t / 1e9, 4), "unit": "GB/s", "cores": cores, "kind": "oracle",
                "sample": f"{reps} full decode steps (all 28 calls each, {t:.1f} s) through the C oracle, "
                          "OpenMP over outputs"}
+        # the same oracle on one thread: an eighth of every call's output columns per step
+        oracle.set_threads(1)
+        try:
+            nb1, t1, reps1 = 0, 0.0, 0
+            while t1 < args.cpu_seconds or reps1 == 0:
+                b_, t_ = cpu_sample(weights, xs, 0.125)
+                nb1, t1, reps1 = nb1 + b_, t1 + t_, reps1 + 1
+        finally:
+            oracle.set_threads(cores)
+        cpu["single_thread"] = {"value": round(nb1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                                "sample": f"{reps1} decode steps over the first eighth of every call's "
+                                          f"output columns ({t1:.1f} s), one thread"}
 
     if args.detail and rank == 0:
         detail(args, sets[0], calls, stream, pk)
@@ -445,6 +458,12 @@ def run_ours(args, world, rank, local):
         del sets, graphs
         torch.cuda.empty_cache()
         prefill = prefill_section(device, stream, pk, weights_cache)
+    quant = None
+    gate_up = None
+    if not args.no_quantize and rank == 0:
+        torch.cuda.empty_cache()
+        quant = quantize_section(device, stream, pk)
+        gate_up = gate_up_section(device, stream, pk)
 
     if rank == 0:
         line = {
@@ -470,6 +489,11 @@ def run_ours(args, world, rank, local):
                 "frac": m2048["frac"], "traffic": None, "peak_source": pk["source"] + " (burst)",
                 "kernel": "w4a16::gm::gemm_kernel", "workload": "M=2048, seven Qwen3-4B projections"}
             line["prefill"] = prefill
+            line["prefill_calls_fields"] = ["M", "projection", "N", "K", "us", "fraction of the bound's measured peak"]
+        if quant is not None:
+            line["quantize"] = quant
+        if gate_up is not None:
+            line["gate_up"] = gate_up
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -543,10 +567,9 @@ def prefill_section(device, stream, pk, weights_cache):
             us = time_calls(make_copy, launch, n_copies, reps, stream)
             del base
             b = algo_bytes(Mo, N, K)
-            rows.append({"M": Mo, "proj": name, "N": N, "K": K, "us": round(us, 3),
-                         "tflops": round(flops / us / 1e6, 2), "gbs": round(b / us / 1e3, 1),
-                         "frac_tensor": round(flops / us / 1e6 / flop_peak, 4),
-                         "frac_hbm": round(b / us / 1e3 / pk["hbm_gbs"], 4)})
+            # compact per-call rows: [M, projection, N, K, us, fraction of the bound's peak]
+            frac = b / us / 1e3 / pk["hbm_gbs"] if key == "lm_head_last_row" else flops / us / 1e6 / flop_peak
+            rows.append([Mo, name, N, K, round(us, 3), round(frac, 4)])
             tot_flops += flops
             tot_us += us
             tot_bytes += b
@@ -559,6 +582,100 @@ def prefill_section(device, stream, pk, weights_cache):
                     "calls": rows}
         torch.cuda.empty_cache()
     return out
+
+
+QUANT_CASES = (("gate 9728 x 2560, FP32", 9728, 2560, "f32"),
+               ("gate 9728 x 2560, BF16", 9728, 2560, "bf16"),
+               ("lm_head 151936 x 2560, BF16", 151936, 2560, "bf16"))
+
+
+def quantize_section(device, stream, pk):
+    """Time the on-GPU quantiser (weights -> packed codes, scales, biases): HBM-bound, its
+    algorithmic bytes are the weights read once and the packed format written once."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    rows, tot_b, tot_us = [], 0, 0.0
+    for desc, N, K, dt in QUANT_CASES:
+        esz = 4 if dt == "f32" else 2
+        b = N * K * esz + N * K // 2 + 4 * N * K // 128
+        g = torch.Generator(device=device).manual_seed(N)
+        base = torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * 0.02
+        if dt == "bf16":
+            base = base.to(torch.bfloat16)
+        n_copies = int(max(2, min(8, math.ceil(2.2 * l2 / b))))
+
+        def make_copy(i, base=base, N=N, K=K):
+            w = base if i == 0 else base.clone()
+            return (w, torch.empty((N, K // 8), dtype=torch.int32, device=device),
+                    torch.empty((N, K // 128), dtype=torch.bfloat16, device=device),
+                    torch.empty((N, K // 128), dtype=torch.bfloat16, device=device))
+
+        def launch(c):
+            w4.w4a16_quantize(c[0], wq=c[1], scales=c[2], biases=c[3])
+
+        us = time_calls(make_copy, launch, n_copies, 16, stream)
+        del base
+        torch.cuda.empty_cache()
+        rows.append([desc, round(us, 3), round(b / us / 1e3, 1), round(b / us / 1e3 / pk["hbm_gbs"], 4)])
+        tot_b += b
+        tot_us += us
+    gbs = tot_b / tot_us / 1e3
+    return {"workload": "W4 g128 min/max quantiser, FP32 or BF16 weights to packed codes, scales and biases",
+            "kernel": "w4a16::qz::quantize_kernel", "bound": "hbm", "us": round(tot_us, 3), "gbs": round(gbs, 1),
+            "frac": round(gbs / pk["hbm_gbs"], 4), "peak": pk["hbm_gbs"], "calls": rows,
+            "calls_fields": ["workload", "us", "GB/s", "fraction of measured HBM"]}
+
+
+def gate_up_section(device, stream, pk):
+    """The fused gate/up projection with SwiGLU (one row-block matvec over interleaved rows)
+    against the same work as two layer calls, Qwen3-4B gate/up 2560 -> 9728, M in {1, 8}."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    N2, K = 9728, 2560
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    gq, gs, gb = synth.make_weights(synth.shape_rng(0, N2, K, seed=11), N2, K)
+    uq, us, ub = synth.make_weights(synth.shape_rng(0, N2, K, seed=12), N2, K)
+
+    def dev(a, bf16):
+        t = torch.from_numpy(a.view(np.int16 if bf16 else np.int32)).to(device)
+        return t.view(torch.bfloat16) if bf16 else t
+
+    fused_w = (dev(synth.interleave_gate_up(gq, uq), False), dev(synth.interleave_gate_up(gs, us), True),
+               dev(synth.interleave_gate_up(gb, ub), True))
+    sep_w = (dev(gq, False), dev(gs, True), dev(gb, True), dev(uq, False), dev(us, True), dev(ub, True))
+    b_w = 2 * algo_bytes(0, N2, K)
+    n_copies = int(max(2, min(8, math.ceil(2.2 * l2 / b_w))))
+    rows = []
+    for M in (1, 8):
+        x = dev(synth.make_x(synth.shape_rng(M, N2, K, seed=13), M, K), True)
+
+        def copy_fused(i, M=M, x=x):
+            w = fused_w if i == 0 else tuple(a.clone() for a in fused_w)
+            return (x,) + w + (torch.empty((M, N2), dtype=torch.bfloat16, device=device),)
+
+        def copy_sep(i, M=M, x=x):
+            w = sep_w if i == 0 else tuple(a.clone() for a in sep_w)
+            return (x,) + w + (torch.empty((M, N2), dtype=torch.bfloat16, device=device),
+                               torch.empty((M, N2), dtype=torch.bfloat16, device=device))
+
+        def fused(c):
+            w4.w4a16_gate_up(c[0], c[1], c[2], c[3], h=c[4])
+
+        def separate(c):
+            w4.w4a16_matmul(c[0], c[1], c[2], c[3], y=c[7])
+            w4.w4a16_matmul(c[0], c[4], c[5], c[6], y=c[8])
+
+        us_f = time_calls(copy_fused, fused, n_copies, 16, stream)
+        us_s = time_calls(copy_sep, separate, n_copies, 16, stream)
+        byts = b_w + 2 * M * K + 2 * M * N2
+        rows.append([M, round(us_f, 3), round(us_s, 3), round(byts / us_f / 1e3, 1),
+                     round(byts / us_f / 1e3 / pk["hbm_gbs"], 4)])
+    torch.cuda.empty_cache()
+    return {"workload": "gate and up 2560 -> 9728 with silu(gate) * up, Qwen3-4B MLP",
+            "kernel": "w4a16::mvr::rows_kernel (gated)", "bound": "hbm", "calls": rows,
+            "calls_fields": ["M", "fused us", "two layer calls us (no SwiGLU)", "fused GB/s",
+                             "fused fraction of measured HBM"]}
 
 
 def profile_case(args, device, stream):
@@ -630,6 +747,7 @@ def main():
                     help="also time every decode call on its own and write the table to PATH (JSON)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the M > 8 measurements")
+    ap.add_argument("--no-quantize", action="store_true", help="skip the quantiser measurement")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="time bound of the CPU baseline sample")
     ap.add_argument("--case", default="", help="profile mode: one problem 'M,N,K' (three eager calls)")
     ap.add_argument("--ref-fraction", type=float, default=0.125,

@@ -33,6 +33,9 @@ PATH_MATVEC = 1
 PATH_GEMM = 2
 PATH_MATVEC_ROWS = 3
 
+DTYPE_F32 = 0
+DTYPE_BF16 = 1
+
 FLAG_NO_PDL = 1
 FLAG_STATIC_WEIGHTS = 2
 FLAG_TEST_DROP_COPY = 4
@@ -78,8 +81,11 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_streamk_owner.argtypes = [i64, i64, i64]
     lib.w4a16_streamk_owner.restype = i64
     lib.w4a16_matvec_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, p]
+    lib.w4a16_quantize.argtypes = [p, ctypes.c_int32, p, p, p, i64, i64, p]
+    lib.w4a16_gate_up.argtypes = [p, p, p, p, p, i64, i64, i64, p]
     for name in ("w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan",
-                 "w4a16_device_status", "w4a16_last_cuda_error", "w4a16_version", "w4a16_matvec_noalloc"):
+                 "w4a16_device_status", "w4a16_last_cuda_error", "w4a16_version", "w4a16_matvec_noalloc",
+                 "w4a16_quantize", "w4a16_gate_up"):
         getattr(lib, name).restype = i32
     return lib
 
@@ -189,6 +195,61 @@ def w4a16_matvec_noalloc(x, wq, scales, biases, y, stream=None):
     return y
 
 
+def interleave_gate_up(gate, up):
+    """Row-interleave a gate and an up tensor [N2, ...] (codes, scales or biases of the two
+    layers) in blocks of 8, the weight layout w4a16_gate_up reads (layout only)."""
+    import torch
+    if gate.shape != up.shape or gate.shape[0] % 8:
+        raise ValueError("gate and up need the same shape and a row count divisible by 8")
+    n2 = gate.shape[0]
+    return torch.stack([gate.reshape(n2 // 8, 8, -1), up.reshape(n2 // 8, 8, -1)], dim=1).reshape(2 * n2, -1)
+
+
+def w4a16_gate_up(x, wq, scales, biases, h=None, stream=None):
+    """Fused gate/up projection, M <= 8: h [M, N2] = bf16(silu(x . gate^T) * (x . up^T)) with the
+    two layers' rows interleaved in blocks of 8 in wq, scales and biases (2 N2 rows)."""
+    import torch
+    M, N, K = _check_tensors(x, wq, scales, biases, h)
+    if N % 16:
+        raise ValueError("the interleaved gate/up rows come in blocks of 16")
+    N2 = N // 2
+    if h is None:
+        h = torch.empty((M, N2), dtype=torch.bfloat16, device=x.device)
+    elif tuple(h.shape) != (M, N2):
+        raise ValueError("h must be [M, N2]")
+    _check(lib.w4a16_gate_up(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(h), M, N2, K,
+                             _stream_handle(stream)), "w4a16_gate_up")
+    return h
+
+
+def w4a16_quantize(w, wq=None, scales=None, biases=None, stream=None):
+    """Quantise weights W [N, K] (float32 or bfloat16, CUDA, contiguous) on the GPU into the
+    packed format: returns (wq int32 [N, K/8], scales bf16 [N, K/128], biases bf16 [N, K/128])."""
+    import torch
+    if w.dim() != 2 or not w.is_cuda or not w.is_contiguous():
+        raise ValueError("w must be a contiguous 2-D CUDA tensor")
+    if w.dtype == torch.float32:
+        dt = DTYPE_F32
+    elif w.dtype == torch.bfloat16:
+        dt = DTYPE_BF16
+    else:
+        raise TypeError("w must be float32 or bfloat16")
+    N, K = w.shape
+    if K % 128:
+        raise W4A16Error(ERR_UNSUPPORTED, "w4a16_quantize")
+    if wq is None:
+        wq = torch.empty((N, K // 8), dtype=torch.int32, device=w.device)
+    if scales is None:
+        scales = torch.empty((N, K // 128), dtype=torch.bfloat16, device=w.device)
+    if biases is None:
+        biases = torch.empty((N, K // 128), dtype=torch.bfloat16, device=w.device)
+    if tuple(wq.shape) != (N, K // 8) or tuple(scales.shape) != (N, K // 128) or tuple(biases.shape) != (N, K // 128):
+        raise ValueError("output shapes must be [N, K/8], [N, K/128], [N, K/128]")
+    _check(lib.w4a16_quantize(_ptr(w), dt, _ptr(wq), _ptr(scales), _ptr(biases), N, K, _stream_handle(stream)),
+           "w4a16_quantize")
+    return wq, scales, biases
+
+
 def w4a16_plan(M: int, N: int, K: int, path=PATH_AUTO, splits=0, workers=0, sm_count=0, row_blocks=0) -> dict:
     opt = make_options(path, splits, workers, sm_count, 0, row_blocks)
     info = PlanInfo()
@@ -215,6 +276,8 @@ def w4a16_streamk_owner(units: int, workers: int, u: int) -> int:
 
 __all__ = [
     "w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan", "w4a16_device_status",
-    "w4a16_release", "w4a16_version", "w4a16_streamk_owner", "w4a16_matvec_noalloc", "status_string", "W4A16Error", "Options",
+    "w4a16_release", "w4a16_version", "w4a16_streamk_owner", "w4a16_matvec_noalloc", "w4a16_quantize",
+    "w4a16_gate_up", "interleave_gate_up",
+    "status_string", "W4A16Error", "Options",
     "PlanInfo", "make_options", "lib", "LIBRARY_PATH",
 ]

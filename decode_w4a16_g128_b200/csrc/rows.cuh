@@ -108,7 +108,17 @@ struct Params {
     long long x_chunk;        // bytes of x this CTA prefetches into L2 (0: none)
     int test_drop_copy;       // tests of the timeout path: CTA 0 never loads its first group's codes
     unsigned long long wait_ns;   // limit of every wait on a copy (kWaitTimeoutNs, shorter in that test)
+    int gated;                // fused gate/up: rows 16 b .. 16 b + 7 are gate rows 8 b .. 8 b + 7, rows
+                              // 16 b + 8 .. 16 b + 15 the up rows of the same outputs; y [M, N / 2] =
+                              // silu(gate) * up; clusters own whole 16-row blocks
+    long long ldy;            // gated: elements between rows of y (a launch may write a column slice)
 };
+
+// silu(g) * u in FP32 (expf of the CUDA math library), then BF16 round to nearest even
+__device__ __forceinline__ uint16_t swiglu_bf16(float g, float u) {
+    const float sg = g / (1.f + expf(-g));
+    return __bfloat16_as_ushort(__float2bfloat16_rn(sg * u));
+}
 
 // BF16 pair (lo, hi) of two words' low / high halves
 __device__ __forceinline__ uint32_t lo_halves(uint32_t a, uint32_t b) { return prmt(a, b, 0x5410u); }
@@ -131,8 +141,10 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
     // this cluster's row blocks; clusters past p.clusters have none (they keep one CTA of
     // every call on each SM, so that the next call's CTAs land one per SM)
     const int cl = static_cast<int>(blockIdx.x) / S;
-    const int hb0 = static_cast<int>(static_cast<long long>(cl) * p.nh / p.clusters);
-    const int nhb = cl < p.clusters ? static_cast<int>(static_cast<long long>(cl + 1) * p.nh / p.clusters) - hb0 : 0;
+    // gated: clusters split the nh / 2 blocks of 16 rows, so that every block pairs gate and up
+    const int unit = p.gated ? 2 : 1, nu = p.nh / unit;
+    const int hb0 = unit * static_cast<int>(static_cast<long long>(cl) * nu / p.clusters);
+    const int nhb = cl < p.clusters ? unit * static_cast<int>(static_cast<long long>(cl + 1) * nu / p.clusters) - hb0 : 0;
     const int nrb = (nhb + 1) / 2;                                       // MMA row blocks (<= RB)
     const long long r0 = 8ll * hb0;                                      // first weight row of the CTA
     const int g0 = static_cast<int>(rank * G / S), g1 = static_cast<int>((rank + 1) * G / S);
@@ -322,21 +334,42 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
     const int tid = threadIdx.x;
     const int RC = 8 * nhb;                      // rows of this CTA
     const int RM = RC * p.M;
-    for (int i = tid; i < RM; i += kWarps * 32) {
-        const int m = i / RC, r = i - m * RC;
+    // the sum of row r (of the CTA) for x row m over the warps, in warp order
+    auto warp_sum = [&](int m, int r) {
         const float *src = red + r * kMaxM + m;   // row block r / 16, row r % 16: offset r * 8
         float v = 0.f;
 #pragma unroll
         for (int ww = 0; ww < kWarps; ++ww) v += src[ww * RB * 16 * kMaxM];
-        if (S == 1) {
-            if (r0 + r < p.N) {
-                if (!isfinite(__bfloat162float(__float2bfloat16_rn(v))))   // not finite: the plain definition
-                    v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8), p.scales + (r0 + r) * G,
-                                     p.biases + (r0 + r) * G, G);
-                p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        return v;
+    };
+    // not finite in FP32 (gated) or BF16: the plain definition of the row's output
+    auto plain_row = [&](int m, long long n) {
+        return plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + n * (p.K / 8), p.scales + n * G,
+                            p.biases + n * G, G);
+    };
+    if (S == 1 && p.gated) {
+        const int JC = RC / 2;                   // outputs per x row: the CTA's gate rows
+        for (int i = tid; i < JC * p.M; i += kWarps * 32) {
+            const int m = i / JC, jl = i - m * JC;
+            const int rg = 16 * (jl >> 3) + (jl & 7), ru = rg + 8;
+            if (r0 + ru >= p.N) continue;
+            float vg = warp_sum(m, rg), vu = warp_sum(m, ru);
+            if (!isfinite(vg)) vg = plain_row(m, r0 + rg);
+            if (!isfinite(vu)) vu = plain_row(m, r0 + ru);
+            p.y[static_cast<long long>(m) * p.ldy + r0 / 2 + jl] = swiglu_bf16(vg, vu);
+        }
+    } else {
+        for (int i = tid; i < RM; i += kWarps * 32) {
+            const int m = i / RC, r = i - m * RC;
+            float v = warp_sum(m, r);
+            if (S == 1) {
+                if (r0 + r < p.N) {
+                    if (!isfinite(__bfloat162float(__float2bfloat16_rn(v)))) v = plain_row(m, r0 + r);
+                    p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+                }
+            } else {
+                part[r * kMaxM + m] = v;
             }
-        } else {
-            part[r * kMaxM + m] = v;
         }
     }
     if (S == 1) return;
@@ -352,15 +385,31 @@ __global__ void __maxnreg__(128) rows_kernel(const __grid_constant__ CUtensorMap
         return;
     }
     const bool parts = mbar_wait_cluster(red_full, 0);   // the other ranks' partial sums landed
-    for (int i = tid; parts && i < RM; i += kWarps * 32) {
-        const int m = i / RC, r = i - m * RC;
+    // the sum of row r for x row m over the ranks, in rank order
+    auto rank_sum = [&](int m, int r) {
         float v = part[r * kMaxM + m];
         for (int s = 1; s < S; ++s) v += slots[((s - 1) * 16 * RB + r) * kMaxM + m];
-        if (r0 + r < p.N) {
-            if (!isfinite(__bfloat162float(__float2bfloat16_rn(v))))   // not finite: the plain definition
-                v = plain_output(p.x + static_cast<long long>(m) * p.K, p.wq + (r0 + r) * (p.K / 8), p.scales + (r0 + r) * G,
-                                 p.biases + (r0 + r) * G, G);
-            p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+        return v;
+    };
+    if (p.gated) {
+        const int JC = RC / 2;
+        for (int i = tid; parts && i < JC * p.M; i += kWarps * 32) {
+            const int m = i / JC, jl = i - m * JC;
+            const int rg = 16 * (jl >> 3) + (jl & 7), ru = rg + 8;
+            if (r0 + ru >= p.N) continue;
+            float vg = rank_sum(m, rg), vu = rank_sum(m, ru);
+            if (!isfinite(vg)) vg = plain_row(m, r0 + rg);
+            if (!isfinite(vu)) vu = plain_row(m, r0 + ru);
+            p.y[static_cast<long long>(m) * p.ldy + r0 / 2 + jl] = swiglu_bf16(vg, vu);
+        }
+    } else {
+        for (int i = tid; parts && i < RM; i += kWarps * 32) {
+            const int m = i / RC, r = i - m * RC;
+            float v = rank_sum(m, r);
+            if (r0 + r < p.N) {
+                if (!isfinite(__bfloat162float(__float2bfloat16_rn(v)))) v = plain_row(m, r0 + r);
+                p.y[static_cast<long long>(m) * p.N + r0 + r] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+            }
         }
     }
 }

@@ -19,6 +19,7 @@
 
 #include "gemm.cuh"
 #include "matvec.cuh"
+#include "quant.cuh"
 #include "rows.cuh"
 
 namespace w4a16 {
@@ -409,9 +410,12 @@ struct RowsChoice {
     int64_t grid = 0;          // CTAs launched (clusters with rows, padded)
 };
 
-bool rows_choose(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, RowsChoice *out) {
+bool rows_choose(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *opt, RowsChoice *out,
+                 bool gated = false) {
     (void)M;
-    const int64_t NH = (N + 7) / 8, G = K / 128;
+    // gated: the unit of the split is a block of 16 rows (a gate half and its up half)
+    const int64_t unit = gated ? 2 : 1;
+    const int64_t NH = (N + 7) / 8, NU = NH / unit, G = K / 128;
     const int req_rb = opt ? opt->row_blocks : 0, req_s = opt ? opt->splits : 0;
     const int order[3] = {1, 2, 4};
     RowsChoice fits[3];
@@ -422,8 +426,8 @@ bool rows_choose(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
         if (s == 0 || s > G) continue;
         const int64_t gcl = (G + s - 1) / s;
         const int64_t slots = std::max<int64_t>(1, sms / s);      // clusters that fit one CTA per SM
-        const int64_t clusters = req_rb ? (NH + 2 * req_rb - 1) / (2 * req_rb) : std::min<int64_t>(slots, NH);
-        const int64_t hb = (NH + clusters - 1) / clusters;
+        const int64_t clusters = req_rb ? (NH + 2 * req_rb - 1) / (2 * req_rb) : std::min<int64_t>(slots, NU);
+        const int64_t hb = unit * ((NU + clusters - 1) / clusters);
         if (mvr::rbs_of(static_cast<int>(std::min<int64_t>(hb, 1 << 20))) > mvr::kMaxRB) continue;
         if (mvr::smem_bytes(static_cast<int>(hb), static_cast<int>(std::min<int64_t>(gcl, 1 << 20)), s) > mvr::kBudget)
             continue;
@@ -518,13 +522,14 @@ cudaError_t rows_launch_rb(const cudaLaunchConfig_t &cfg, const CUtensorMap &tm_
 }
 
 int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void *stream, bool pdl,
-                bool static_weights, bool test_drop_copy) {
+                bool static_weights, bool test_drop_copy, bool gated = false, int64_t ldy = 0) {
     const int G = static_cast<int>(p.K / 128);
     const int rb = pl.row_blocks, S = pl.splits;
     if (rb < 1 || rb > mvr::kMaxRB || S < 1 || S > mvr::kMaxSplits) return W4A16_ERR_INVALID_ARG;
     const int64_t NH = (p.N + 7) / 8;
+    const int64_t unit = gated ? 2 : 1, NU = NH / unit;
     const int clusters = static_cast<int>(pl.tiles);
-    const int hb_lo = static_cast<int>(NH / clusters), hb_hi = static_cast<int>((NH + clusters - 1) / clusters);
+    const int hb_lo = static_cast<int>(unit * (NU / clusters)), hb_hi = static_cast<int>(unit * ((NU + clusters - 1) / clusters));
     if (mvr::rbs_of(hb_hi) != rb) return W4A16_ERR_INVALID_ARG;
     CUtensorMap tm_hi, tm_lo;
     // codes: [N, K/8] uint32, boxes of one group (16 words = 64 B) x the cluster's rows (8 hb_hi,
@@ -554,6 +559,8 @@ int launch_rows(DeviceInfo *d, const Problem &p, const w4a16_plan_info &pl, void
     kp.hb_hi = hb_hi;
     kp.static_weights = static_weights ? 1 : 0;
     kp.test_drop_copy = test_drop_copy ? 1 : 0;
+    kp.gated = gated ? 1 : 0;
+    kp.ldy = ldy > 0 ? ldy : p.N / 2;
     kp.wait_ns = test_drop_copy ? 200000ull : kWaitTimeoutNs;
     // every CTA prefetches an equal 16-byte-aligned share of x into L2 before the wait
     const long long xbytes = p.M * p.K * 2;
@@ -940,6 +947,90 @@ int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u) {
 int w4a16_matvec_noalloc(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *y,
                          int64_t M, int64_t N, int64_t K, void *stream) {
     return noalloc_matvec(Problem{x, wq, scales, biases, y, M, N, K}, stream);
+}
+
+int w4a16_gate_up(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *h, int64_t M,
+                  int64_t N2, int64_t K, void *stream) {
+    if (M < 0 || N2 < 0 || K < 0) return W4A16_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N2 % 8 != 0 || M > mvr::kMaxM || N2 >= (int64_t(1) << 30) || K >= (int64_t(1) << 31))
+        return W4A16_ERR_UNSUPPORTED;
+    if (M == 0 || N2 == 0) return W4A16_OK;
+    if (!h) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(h)) return W4A16_ERR_MISALIGNED;
+    const int64_t N = 2 * N2;
+    if (K == 0) {   // an empty sum: silu(0) * 0 = +0 everywhere
+        cudaError_t e = cudaMemsetAsync(h, 0, size_t(M) * N2 * 2, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+    }
+    if (!x || !wq || !scales || !biases) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(wq) || !aligned16(scales) || !aligned16(biases)) return W4A16_ERR_MISALIGNED;
+    const size_t nh = size_t(M) * N2 * 2;
+    if (overlaps(h, nh, x, size_t(M) * K * 2) || overlaps(h, nh, wq, size_t(N) * K / 2) ||
+        overlaps(h, nh, scales, size_t(N) * (K / 128) * 2) || overlaps(h, nh, biases, size_t(N) * (K / 128) * 2))
+        return W4A16_ERR_INVALID_ARG;
+    int dev = 0;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo *d = nullptr;
+    rc = device_setup(dev, &d);
+    if (rc) return rc;
+    // A CTA holds all of its rows' codes: where the 2 N2 rows exceed what the SMs hold at once,
+    // the outputs are cut into column slices of whole 16-row blocks, one launch each (the later
+    // ones fetch their weights while the one before finishes).
+    const int64_t nb = N2 / 8, G = K / 128;
+    int64_t chunks = 0;
+    RowsChoice c;
+    for (int64_t t = 1; t <= 64 && t <= nb && !chunks; ++t)
+        if (rows_choose(M, 16 * ((nb + t - 1) / t), K, d->sms, nullptr, &c, true)) chunks = t;
+    if (!chunks) return W4A16_ERR_UNSUPPORTED;
+    for (int64_t i = 0; i < chunks; ++i) {
+        const int64_t b0 = i * nb / chunks, b1 = (i + 1) * nb / chunks, rows = 16 * (b1 - b0);
+        if (rows == 0) continue;
+        if (!rows_choose(M, rows, K, d->sms, nullptr, &c, true)) return W4A16_ERR_UNSUPPORTED;
+        w4a16_plan_info pl;
+        plan_rows(rows, K, c, &pl);
+        const Problem sub{x, wq + 16 * b0 * (K / 8), static_cast<const uint16_t *>(scales) + 16 * b0 * G,
+                          static_cast<const uint16_t *>(biases) + 16 * b0 * G, static_cast<uint16_t *>(h) + 8 * b0,
+                          M, rows, K};
+        rc = launch_rows(d, sub, pl, stream, true, i > 0, false, true, N2);
+        if (rc) return rc;
+    }
+    return W4A16_OK;
+}
+
+int w4a16_quantize(const void *w, int32_t w_dtype, uint32_t *wq, void *scales, void *biases, int64_t N, int64_t K,
+                   void *stream) {
+    if (N < 0 || K < 0 || (w_dtype != W4A16_DTYPE_F32 && w_dtype != W4A16_DTYPE_BF16)) return W4A16_ERR_INVALID_ARG;
+    if (K % 128 != 0 || N >= (int64_t(1) << 31) || K >= (int64_t(1) << 31)) return W4A16_ERR_UNSUPPORTED;
+    if (N == 0 || K == 0) return W4A16_OK;
+    if (!w || !wq || !scales || !biases) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(w) || !aligned16(wq) || !aligned16(scales) || !aligned16(biases)) return W4A16_ERR_MISALIGNED;
+    const size_t nw = size_t(N) * K * (w_dtype == W4A16_DTYPE_F32 ? 4 : 2);
+    const size_t nq = size_t(N) * K / 2, ns = size_t(N) * (K / 128) * 2;
+    if (overlaps(w, nw, wq, nq) || overlaps(w, nw, scales, ns) || overlaps(w, nw, biases, ns) ||
+        overlaps(wq, nq, scales, ns) || overlaps(wq, nq, biases, ns) || overlaps(scales, ns, biases, ns))
+        return W4A16_ERR_INVALID_ARG;
+    int dev = 0;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo *d = nullptr;
+    rc = device_setup(dev, &d);
+    if (rc) return rc;
+    // (row, group) pairs, four per warp, eight warps per CTA, at most eight CTAs per SM
+    const int64_t pairs = N * (K / 128);
+    const int64_t per_cta = int64_t(qz::kWarps) * qz::kPairsPerWarp;
+    const int64_t grid = std::max<int64_t>(1, std::min<int64_t>((pairs + per_cta - 1) / per_cta, int64_t(d->sms) * 8));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (w_dtype == W4A16_DTYPE_BF16)
+        qz::quantize_kernel<true><<<static_cast<unsigned>(grid), qz::kThreads, 0, st>>>(
+            w, wq, static_cast<uint16_t *>(scales), static_cast<uint16_t *>(biases), N, static_cast<int>(K));
+    else
+        qz::quantize_kernel<false><<<static_cast<unsigned>(grid), qz::kThreads, 0, st>>>(
+            w, wq, static_cast<uint16_t *>(scales), static_cast<uint16_t *>(biases), N, static_cast<int>(K));
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
 }
 
 }  // extern "C"

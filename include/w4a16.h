@@ -213,8 +213,8 @@ int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u);
  * W4A16_ERR_UNSUPPORTED without launching.  Other arguments, layouts and
  * errors are those of w4a16_matmul.
  * Set-up: the first call on a device looks up the array's device address
- * (cudaGetSymbolAddress); make that first call before any stream capture.
- * w4a16_release forgets the address; call it before resetting a device.
+ * (cudaGetSymbolAddress).  w4a16_release forgets the address; call it before
+ * resetting a device.
  * Sharing: every call uses the same array and clears its tickets on `stream`
  * before launching, so calls whose kernels can overlap on the GPU (different
  * streams without ordering) race and give undefined results; serialise them.
@@ -226,6 +226,60 @@ int64_t w4a16_streamk_owner(int64_t units, int64_t workers, int64_t u);
 int w4a16_matvec_noalloc(const void *x, const uint32_t *wq, const void *scales,
                          const void *biases, void *y, int64_t M, int64_t N,
                          int64_t K, void *stream);
+
+/*
+ * Fused gate/up projection with the SwiGLU product (decode, M <= 8):
+ *   h[m, j] = bf16_rne(silu(g[m, j]) * u[m, j]),  silu(g) = g / (1 + exp(-g)),
+ * where g and u are the FP32 sums of two W4A16 layers over the same x (the gate
+ * and up projections of a gated MLP), never rounded to BF16 in between.  Both
+ * share x, so one pass of the row-block matvec reads x once and writes h
+ * (llama.cpp issue "Metal prefill speedup (~68%) on M5 Max": SwiGLU fused into
+ * the matrix product; its related work fuses gate/up with interleaved rows).
+ *
+ * Weights: the two layers' rows interleaved in blocks of 8: rows 16 b .. 16 b + 7
+ * of wq, scales and biases are gate rows 8 b .. 8 b + 7 and rows 16 b + 8 .. 16 b
+ * + 15 the up rows 8 b .. 8 b + 7 (2 N2 rows in all, each in the packed format
+ * above).  x bf16 [M, K]; h bf16 [M, N2], written.  Sizes: 0 <= M <= 8, N2 % 8
+ * == 0, K % 128 == 0, else W4A16_ERR_UNSUPPORTED; M == 0 or N2 == 0 launches
+ * nothing.  Alignment, aliasing, ownership and stream semantics as w4a16_matmul.
+ * A gate or up sum that is not finite in FP32 is recomputed by the plain
+ * definition, as in w4a16_matmul.
+ */
+int w4a16_gate_up(const void *x, const uint32_t *wq, const void *scales,
+                  const void *biases, void *h, int64_t M, int64_t N2, int64_t K,
+                  void *stream);
+
+/*
+ * Quantiser: weights W [N, K] -> the packed format above (wq [N, K/8] codes,
+ * scales and biases [N, K/128] BF16), on the GPU.
+ *
+ * The recipe is the affine min/max quantisation per 128-group that the
+ * layer's weights are defined with (tiny-llm "Week 2 Day 6", Task 3: one
+ * scale and bias per group; the reference problem's inputs: scale = (max -
+ * min) / 15, bias = min, q rounded and clamped to 0..15, eight codes per
+ * uint32 low nibble first).  Per row n and group g, all in FP32:
+ *   lo, hi = min, max of the group's 128 values (a zero is taken as +0)
+ *   scale  = bf16_rne((hi - lo) / 15)       bias = bf16_rne(lo)
+ *   q[k]   = 0 when scale == 0 (a constant group), else
+ *            clamp(rint((w[k] - bias) / scale), 0, 15), with the BF16
+ *            scale and bias, IEEE division and rint rounding half to even.
+ * Each step is correctly rounded: the output is bit-identical to the same
+ * recipe computed sequentially on a CPU.  Inputs must be finite.
+ *
+ * Arguments: w device pointer to W, row-major FP32 (w_dtype = W4A16_DTYPE_F32)
+ * or BF16 (W4A16_DTYPE_BF16); wq, scales, biases device pointers to the
+ * outputs, written; N, K sizes with K % 128 == 0 (else W4A16_ERR_UNSUPPORTED);
+ * N == 0 or K == 0 returns W4A16_OK and launches nothing.  Every pointer must
+ * be 16-byte aligned (W4A16_ERR_MISALIGNED) and the outputs must not overlap
+ * w (W4A16_ERR_INVALID_ARG).  Ownership and stream semantics as w4a16_matmul:
+ * the work is enqueued on `stream` and the call returns without waiting.
+ */
+enum w4a16_dtype {
+    W4A16_DTYPE_F32 = 0,
+    W4A16_DTYPE_BF16 = 1
+};
+int w4a16_quantize(const void *w, int32_t w_dtype, uint32_t *wq, void *scales,
+                   void *biases, int64_t N, int64_t K, void *stream);
 
 #ifdef __cplusplus
 }

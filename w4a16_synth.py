@@ -220,3 +220,14 @@ def make_overflow_problem(M: int, N: int, K: int, sign: float = 1.0, exponent: i
         W = np.float32(0.05) + np.abs(W)
     wq, s, b = quantize_w4_g128(W)
     return {"x": x, "wq": wq, "scales": s, "biases": b, "M": M, "N": N, "K": K}
+
+
+def interleave_gate_up(gate, up):
+    """Row-interleave two [N2, ...] arrays (a packed layer's codes, scales or biases) in blocks
+    of 8 for the fused gate/up projection: gate rows 8 b .. 8 b + 7, then up rows 8 b .. 8 b + 7
+    (a layout only, no arithmetic)."""
+    gate, up = np.asarray(gate), np.asarray(up)
+    if gate.shape != up.shape or gate.shape[0] % 8:
+        raise ValueError("gate and up need the same shape and a row count divisible by 8")
+    n2 = gate.shape[0]
+    return np.stack([gate.reshape(n2 // 8, 8, -1), up.reshape(n2 // 8, 8, -1)], axis=1).reshape(2 * n2, -1)
