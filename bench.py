@@ -679,9 +679,39 @@ def gate_up_section(device, stream, pk):
 
 
 def profile_case(args, device, stream):
-    """Three eager calls of one M x N x K problem (for an ncu capture of one kernel)."""
+    """Three eager calls of one problem (for an ncu capture of one kernel): 'M,N,K' (the layer),
+    'quant:N,K,f32|bf16' (the quantiser) or 'gateup:M,N2,K' (the fused gate/up projection)."""
     import torch
     import decode_w4a16_g128_b200 as w4
+    if args.case.startswith("quant:"):
+        n_, k_, dt = args.case[len("quant:"):].split(",")
+        N, K = int(n_), int(k_)
+        g = torch.Generator(device=device).manual_seed(N)
+        W = torch.randn((N, K), generator=g, device=device, dtype=torch.float32) * 0.02
+        if dt == "bf16":
+            W = W.to(torch.bfloat16)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                w4.w4a16_quantize(W)
+        torch.cuda.synchronize()
+        return 0
+    if args.case.startswith("gateup:"):
+        M, N2, K = (int(v) for v in args.case[len("gateup:"):].split(","))
+        rng = synth.shape_rng(M, N2, K, seed=3)
+        x = synth.make_x(rng, M, K)
+        gw = [synth.make_weights(rng, N2, K) for _ in range(2)]
+        gu = [synth.interleave_gate_up(gw[0][i], gw[1][i]) for i in range(3)]
+        xd = torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16)
+        wd = torch.from_numpy(gu[0].view(np.int32)).to(device)
+        sd = torch.from_numpy(gu[1].view(np.int16)).to(device).view(torch.bfloat16)
+        bd = torch.from_numpy(gu[2].view(np.int16)).to(device).view(torch.bfloat16)
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                w4.w4a16_gate_up(xd, wd, sd, bd)
+        torch.cuda.synchronize()
+        if w4.w4a16_device_status(stream) != w4.OK:
+            raise RuntimeError("device status not ok")
+        return 0
     M, N, K = (int(v) for v in args.case.split(","))
     prob = synth.make_problem(M, N, K)
     d = [torch.from_numpy(prob[k].view(np.int16 if prob[k].dtype == np.uint16 else np.int32)).to(device)
