@@ -460,10 +460,13 @@ def run_ours(args, world, rank, local):
         prefill = prefill_section(device, stream, pk, weights_cache)
     quant = None
     gate_up = None
+    skinny = None
     if not args.no_quantize and rank == 0:
         torch.cuda.empty_cache()
         quant = quantize_section(device, stream, pk)
         gate_up = gate_up_section(device, stream, pk)
+    if not args.no_prefill and rank == 0:
+        skinny = skinny_section(device, stream, pk, weights_cache)
 
     if rank == 0:
         line = {
@@ -494,6 +497,8 @@ def run_ours(args, world, rank, local):
             line["quantize"] = quant
         if gate_up is not None:
             line["gate_up"] = gate_up
+        if skinny is not None:
+            line["skinny"] = skinny
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -676,6 +681,41 @@ def gate_up_section(device, stream, pk):
             "kernel": "w4a16::mvr::rows_kernel (gated)", "bound": "hbm", "calls": rows,
             "calls_fields": ["M", "fused us", "two layer calls us (no SwiGLU)", "fused GB/s",
                              "fused fraction of measured HBM"]}
+
+
+def skinny_section(device, stream, pk, weights_cache):
+    """8 < M <= 32: slices of the row-block matvec against the GEMM, per Qwen3-4B projection
+    (the measured crossover behind the automatic choice)."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    rows = []
+    for M in (12, 16, 24, 32):
+        for (name, K, N) in synth.QWEN3_4B_PROJECTIONS:
+            if (name, K, N) not in weights_cache:
+                weights_cache[(name, K, N)] = synth.make_weights(synth.shape_rng(0, N, K, seed=0), N, K)
+            wq, sc, bi = weights_cache[(name, K, N)]
+            x = synth.make_x(synth.shape_rng(M, N, K, seed=1), M, K)
+            base = (torch.from_numpy(x.view(np.int16)).to(device).view(torch.bfloat16),
+                    torch.from_numpy(wq.view(np.int32)).to(device),
+                    torch.from_numpy(sc.view(np.int16)).to(device).view(torch.bfloat16),
+                    torch.from_numpy(bi.view(np.int16)).to(device).view(torch.bfloat16))
+            n_copies = int(max(2, min(16, math.ceil(2.2 * l2 / algo_bytes(M, N, K)))))
+
+            def make_copy(i, base=base, M=M, N=N):
+                t = base if i == 0 else tuple(a.clone() for a in base)
+                return t + (torch.empty((M, N), dtype=torch.bfloat16, device=device),)
+
+            res = []
+            for path in (w4.PATH_MATVEC_ROWS, w4.PATH_GEMM):
+                def launch(c, path=path):
+                    w4.w4a16_matmul_ex(c[0], c[1], c[2], c[3], y=c[4], path=path)
+                res.append(time_calls(make_copy, launch, n_copies, 16, stream))
+            del base
+            rows.append([M, name, N, K, round(res[0], 3), round(res[1], 3)])
+    torch.cuda.empty_cache()
+    return {"workload": "M in {12, 16, 24, 32} x the seven Qwen3-4B projections",
+            "calls": rows, "calls_fields": ["M", "projection", "N", "K", "row-block slices us", "GEMM us"]}
 
 
 def profile_case(args, device, stream):

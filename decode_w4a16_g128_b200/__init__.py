@@ -58,7 +58,7 @@ class PlanInfo(ctypes.Structure):
                 ("grid_y", ctypes.c_int32), ("grid_z", ctypes.c_int32), ("block", ctypes.c_int32),
                 ("smem_bytes", ctypes.c_int32), ("cluster", ctypes.c_int32), ("tiles", ctypes.c_int64),
                 ("units", ctypes.c_int64), ("workspace_bytes", ctypes.c_int64), ("row_blocks", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("slices", ctypes.c_int32)]
 
 
 def _load() -> ctypes.CDLL:

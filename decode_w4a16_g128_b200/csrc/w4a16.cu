@@ -27,6 +27,7 @@ namespace {
 
 constexpr int kVersion = 100;          // 0.1.0
 constexpr int kMinTickets = 1 << 16;   // ticket slots allocated up front (grows on demand)
+constexpr int kSkinnyMaxM = 32;        // the row-block matvec over slices of 8 x rows, up to this M
 // Shared memory of a matvec CTA: one CTA per SM, most of the SM's shared
 // memory, so that the copy ring is deep enough to cover HBM latency.
 constexpr long long kMatvecBudget = 220 * 1024;
@@ -271,7 +272,7 @@ int choose_path(int64_t M, const w4a16_options *opt, int *path) {
     } else if (req == W4A16_PATH_GEMM) {
         *path = W4A16_PATH_GEMM;
     } else if (req == W4A16_PATH_MATVEC_ROWS) {
-        if (M > mvr::kMaxM) return W4A16_ERR_UNSUPPORTED;
+        if (M > kSkinnyMaxM) return W4A16_ERR_UNSUPPORTED;
         *path = W4A16_PATH_MATVEC_ROWS;
     } else {
         return W4A16_ERR_INVALID_ARG;
@@ -452,9 +453,10 @@ bool rows_choose(int64_t M, int64_t N, int64_t K, int sms, const w4a16_options *
     return true;
 }
 
-void plan_rows(int64_t N, int64_t K, const RowsChoice &c, w4a16_plan_info *pl) {
+void plan_rows(int64_t N, int64_t K, const RowsChoice &c, w4a16_plan_info *pl, int64_t M = 1) {
     const int64_t G = K / 128;
     std::memset(pl, 0, sizeof(*pl));
+    pl->slices = static_cast<int32_t>(std::max<int64_t>(1, (M + mvr::kMaxM - 1) / mvr::kMaxM));
     pl->path = W4A16_PATH_MATVEC_ROWS;
     pl->splits = c.splits;
     pl->grid_x = static_cast<int32_t>(c.grid);
@@ -468,20 +470,33 @@ void plan_rows(int64_t N, int64_t K, const RowsChoice &c, w4a16_plan_info *pl) {
     pl->workspace_bytes = 0;
 }
 
+// The automatic choice for 8 < M <= 32 (measured on B200, back-to-back calls of the Qwen3-4B
+// projections): two slices of the row-block matvec beat the GEMM on every projection.
+bool skinny_prefers_rows(int64_t M, int64_t N, int64_t K) {
+    (void)N;
+    (void)K;
+    return (M + mvr::kMaxM - 1) / mvr::kMaxM <= 2;
+}
+
 // max_splits: the GEMM's largest K split on this device (forced splits above it are refused)
 int plan(int64_t M, int64_t N, int64_t K, const w4a16_options *opt, int sms, int max_splits, w4a16_plan_info *pl) {
     int path = 0;
     int rc = choose_path(M, opt, &path);
     if (rc) return rc;
     const int req = opt ? opt->path : W4A16_PATH_AUTO;
+    // 8 < M <= 32 on the automatic path: slices of the row-block matvec where the measured
+    // crossover against the GEMM (whose tiles pad M to 128) says so
+    const bool skinny = req == W4A16_PATH_AUTO && M > mvr::kMaxM && M <= kSkinnyMaxM &&
+                        !(opt && (opt->splits > 0 || opt->workers > 0)) && skinny_prefers_rows(M, N, K);
     RowsChoice rc_rows;
-    const bool rows_fit = path == W4A16_PATH_MATVEC_ROWS || path == W4A16_PATH_MATVEC
+    const bool rows_fit = path == W4A16_PATH_MATVEC_ROWS || path == W4A16_PATH_MATVEC || skinny
                               ? rows_choose(M, N, K, sms, opt, &rc_rows) : false;
     if (path == W4A16_PATH_MATVEC_ROWS && !rows_fit) return W4A16_ERR_UNSUPPORTED;
     if (path == W4A16_PATH_MATVEC && req == W4A16_PATH_AUTO && !(opt && opt->workers > 0) && rows_fit)
         path = W4A16_PATH_MATVEC_ROWS;
+    if (skinny && rows_fit) path = W4A16_PATH_MATVEC_ROWS;
     if (path == W4A16_PATH_MATVEC_ROWS) {
-        plan_rows(N, K, rc_rows, pl);
+        plan_rows(N, K, rc_rows, pl, M);
         return W4A16_OK;
     }
     if (path == W4A16_PATH_MATVEC) {
@@ -754,8 +769,19 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     const bool pdl = !(opt && (opt->flags & W4A16_FLAG_NO_PDL));
     const bool static_weights = opt && (opt->flags & W4A16_FLAG_STATIC_WEIGHTS);
     const bool drop = opt && (opt->flags & W4A16_FLAG_TEST_DROP_COPY);
-    if (drop && pl.path != W4A16_PATH_MATVEC_ROWS) return W4A16_ERR_INVALID_ARG;
-    if (pl.path == W4A16_PATH_MATVEC_ROWS) return launch_rows(d, p, pl, stream, pdl, pdl && static_weights, drop);
+    if (drop && (pl.path != W4A16_PATH_MATVEC_ROWS || p.M > mvr::kMaxM)) return W4A16_ERR_INVALID_ARG;
+    if (pl.path == W4A16_PATH_MATVEC_ROWS) {
+        // one launch per slice of 8 x rows; each slice after the first reads the weights the one
+        // before has just brought into L2, and fetches them before its dependency wait
+        for (int64_t m0 = 0; m0 < p.M; m0 += mvr::kMaxM) {
+            const int64_t mi = std::min<int64_t>(mvr::kMaxM, p.M - m0);
+            const Problem sub{static_cast<const uint16_t *>(p.x) + m0 * p.K, p.wq, p.scales, p.biases,
+                              static_cast<uint16_t *>(p.y) + m0 * p.N, mi, p.N, p.K};
+            rc = launch_rows(d, sub, pl, stream, pdl, pdl && (static_weights || m0 > 0), drop);
+            if (rc) return rc;
+        }
+        return W4A16_OK;
+    }
     if (pl.path == W4A16_PATH_MATVEC) {
         Workspace *ws = nullptr;
         rc = workspace_get(dev, stream, size_t(pl.grid_x) * mv::kPartialFloats, pl.tiles, &ws);

@@ -65,13 +65,18 @@ enum w4a16_path {
     W4A16_PATH_AUTO = 0,        /* M <= 8: matvec; M > 8: tensor-core GEMM (Task 1 dispatch rule) */
     W4A16_PATH_MATVEC = 1,      /* weight-streaming matvec, M <= 8 only                           */
     W4A16_PATH_GEMM = 2,        /* tcgen05 tensor-core GEMM, any M >= 1                            */
-    W4A16_PATH_MATVEC_ROWS = 3  /* row-block matvec, M <= 8: a CTA holds all codes, scales and biases
+    W4A16_PATH_MATVEC_ROWS = 3  /* row-block matvec, M <= 32: a CTA holds all codes, scales and biases
                                    of 16 x row_blocks weight rows over a K range in shared memory
                                    (the whole of K, or 1/splits of it with the splits of a row range
                                    added in a thread-block cluster); two CTAs fit on an SM.  Only
-                                   where such a split fits (else W4A16_ERR_UNSUPPORTED).
+                                   where such a split fits (else W4A16_ERR_UNSUPPORTED).  For
+                                   8 < M <= 32 it runs once per slice of 8 x rows (ceil(M / 8)
+                                   launches; the later ones find the weights in L2 and fetch them
+                                   while the one before finishes).
                                    W4A16_PATH_AUTO takes it for M <= 8 when it fits and no worker
-                                   count is given, the stream-K matvec (W4A16_PATH_MATVEC) otherwise */
+                                   count is given, the stream-K matvec (W4A16_PATH_MATVEC) otherwise;
+                                   for 8 < M <= 32 it takes it where the measured crossover against
+                                   the GEMM says so (w4a16_plan reports the choice)             */
 };
 
 /*
@@ -159,7 +164,8 @@ typedef struct w4a16_plan_info {
                                 row-block matvec: 16-row blocks                         */
     int64_t workspace_bytes; /* library workspace the call needs                        */
     int32_t row_blocks;      /* row-block matvec: blocks of 16 weight rows per cluster   */
-    int32_t reserved;
+    int32_t slices;          /* row-block matvec: launches over slices of 8 x rows (1 for
+                                M <= 8, ceil(M / 8) for 8 < M <= 32); 0 on other paths   */
 } w4a16_plan_info;
 
 /*

@@ -106,12 +106,31 @@ def test_row_block_split_limit():
 
 def test_dispatch_rule():
     """M <= 8 streams weights through a matvec (the row-block one where a CTA's whole rows
-    fit, the stream-K one otherwise); larger M goes to the tensor-core GEMM."""
+    fit, the stream-K one otherwise); 8 < M <= 16 takes two slices of the row-block matvec
+    where it fits (the measured crossover against the GEMM), larger M the tensor-core GEMM."""
     for M in range(1, 9):
-        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148)["path"] == w4.PATH_MATVEC_ROWS
+        pl = w4.w4a16_plan(M, 4096, 2560, sm_count=148)
+        assert pl["path"] == w4.PATH_MATVEC_ROWS and pl["slices"] == 1
         assert w4.w4a16_plan(M, 151936, 2560, sm_count=148)["path"] == w4.PATH_MATVEC
         assert w4.w4a16_plan(M, 4096, 2560, sm_count=148, workers=64)["path"] == w4.PATH_MATVEC
-    assert w4.w4a16_plan(9, 4096, 2560, sm_count=148)["path"] == w4.PATH_GEMM
+    for M in range(9, 17):
+        pl = w4.w4a16_plan(M, 4096, 2560, sm_count=148)
+        assert pl["path"] == w4.PATH_MATVEC_ROWS and pl["slices"] == 2
+        assert w4.w4a16_plan(M, 151936, 2560, sm_count=148)["path"] == w4.PATH_GEMM   # rows do not fit
+        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148, splits=2)["path"] == w4.PATH_GEMM
+    for M in (17, 32, 33, 128):
+        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148)["path"] == w4.PATH_GEMM
+        assert w4.w4a16_plan(M, 4096, 2560, sm_count=148)["slices"] == 0
+
+
+def test_row_block_slices():
+    """The row-block path runs ceil(M / 8) slices of 8 x rows, up to M = 32."""
+    for M, sl in ((9, 2), (24, 3), (25, 4), (32, 4)):
+        pl = w4.w4a16_plan(M, 2560, 9728, path=w4.PATH_MATVEC_ROWS, sm_count=148)
+        assert pl["path"] == w4.PATH_MATVEC_ROWS and pl["slices"] == sl
+    with pytest.raises(w4.W4A16Error) as e:
+        w4.w4a16_plan(33, 2560, 9728, path=w4.PATH_MATVEC_ROWS, sm_count=148)
+    assert e.value.status == w4.ERR_UNSUPPORTED
 
 
 def rows_smem(hb, gcl, s):
@@ -151,8 +170,8 @@ def test_rows_plan_limits():
     with pytest.raises(w4.W4A16Error) as e:
         w4.w4a16_plan(1, 151936, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148)
     assert e.value.status == w4.ERR_UNSUPPORTED
-    with pytest.raises(w4.W4A16Error) as e:
-        w4.w4a16_plan(9, 4096, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148)
+    with pytest.raises(w4.W4A16Error) as e:   # at most four slices of 8 x rows
+        w4.w4a16_plan(33, 4096, 2560, path=w4.PATH_MATVEC_ROWS, sm_count=148)
     assert e.value.status == w4.ERR_UNSUPPORTED
     # K = 9728 without a split would need 2 row blocks x 76 groups: more than half an SM
     assert rows_smem(4, 76, 1) > 115712 >= rows_smem(5, 38, 2)
