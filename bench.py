@@ -55,6 +55,9 @@ DECODE_KERNEL = "w4a16::mvr::rows_kernel"
 KERNEL_SOURCES = ("decode_w4a16_g128_b200/csrc/rows.cuh", "decode_w4a16_g128_b200/csrc/ptx.cuh",
                   "decode_w4a16_g128_b200/csrc/plain.cuh")
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "rows_decode_traffic.txt")
+GEMM_SOURCES = ("decode_w4a16_g128_b200/csrc/gemm.cuh", "decode_w4a16_g128_b200/csrc/ptx.cuh",
+                "decode_w4a16_g128_b200/csrc/plain.cuh")
+GEMM_TRAFFIC_FILE = os.path.join(ROOT, "profiles", "gemm_m2048_gate_traffic.txt")
 
 
 def algo_bytes(M, N, K):
@@ -91,21 +94,21 @@ def peaks():
         return dict(FALLBACK_PEAKS, source="fallback")
 
 
-def kernel_hash():
+def kernel_hash(sources=KERNEL_SOURCES):
     h = hashlib.sha256()
-    for rel in KERNEL_SOURCES:
+    for rel in sources:
         with open(os.path.join(ROOT, rel), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
 
-def recorded_traffic():
+def recorded_traffic(path=TRAFFIC_FILE, sources=KERNEL_SOURCES):
     """Per-launch DRAM bytes from the committed ncu capture, if it matches this kernel."""
     try:
-        with open(TRAFFIC_FILE) as f:
+        with open(path) as f:
             d = dict(line.split(":", 1) for line in f if ":" in line and not line.startswith("#"))
         d = {k.strip(): v.strip() for k, v in d.items()}
-        if d.get("kernel_sha") != kernel_hash():
+        if d.get("kernel_sha") != kernel_hash(sources):
             return None
         return int(d["dram_bytes_per_launch"])
     except (OSError, ValueError, KeyError):
@@ -489,7 +492,9 @@ def run_ours(args, world, rank, local):
             m2048 = prefill["prefill_m2048"]
             line["roofline_gemm"] = {
                 "bound": "tensor", "achieved": m2048["tflops"], "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                "frac": m2048["frac"], "traffic": None, "peak_source": pk["source"] + " (burst)",
+                "frac": m2048["frac"], "traffic": recorded_traffic(GEMM_TRAFFIC_FILE, GEMM_SOURCES),
+                "traffic_launch": "gate, M=2048 (DRAM bytes of one launch; most of y is still in L2 when it ends)",
+                "peak_source": pk["source"] + " (burst)",
                 "kernel": "w4a16::gm::gemm_kernel", "workload": "M=2048, seven Qwen3-4B projections"}
             line["prefill"] = prefill
             line["prefill_calls_fields"] = ["M", "projection", "N", "K", "us", "fraction of the bound's measured peak"]
