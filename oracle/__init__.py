@@ -69,6 +69,10 @@ class Oracle:
         lib.w4a16_oracle_set_threads.restype = None
         lib.w4a16_oracle_gate_up.argtypes = [p, p, p, p, p, i64, i64, i64]
         lib.w4a16_oracle_gate_up.restype = ctypes.c_int
+        lib.w4a16_oracle_matmul_bits.argtypes = [p, p, p, p, p, i64, i64, i64, ctypes.c_int]
+        lib.w4a16_oracle_matmul_bits.restype = ctypes.c_int
+        lib.w4a16_oracle_unpack_bits.argtypes = [p, p, i64, i64, ctypes.c_int]
+        lib.w4a16_oracle_unpack_bits.restype = ctypes.c_int
         for name in ("w4a16_oracle_quantize", "w4a16_oracle_quantize_bf16"):
             fn = getattr(lib, name)
             fn.argtypes = [p, p, p, p, i64, i64]
@@ -104,6 +108,30 @@ class Oracle:
         if self.lib.w4a16_oracle_matmul_f32(*ptrs, acc.ctypes.data_as(ctypes.c_void_p), M, N, K):
             raise ValueError("oracle rejected its arguments")
         return acc
+
+    def matmul_bits(self, x, wq, scales, biases, bits: int) -> np.ndarray:
+        """y [M,N] BF16 bits with b-bit codes (wq [N, K b / 32], 32 / b codes per word, low first)."""
+        x, px = _c(x, np.uint16)
+        wq, pw = _c(wq, np.uint32)
+        s, ps = _c(scales, np.uint16)
+        b, pb = _c(biases, np.uint16)
+        M, K = x.shape
+        N = wq.shape[0]
+        G = K // 128 if K % 128 == 0 else -1
+        if bits not in (2, 4, 8) or wq.shape != (N, K * bits // 32) or s.shape != (N, G) or b.shape != (N, G):
+            raise ValueError("shape mismatch between x, wq, scales and biases (or bits not 2, 4, 8)")
+        y = np.empty((M, N), dtype=np.uint16)
+        if self.lib.w4a16_oracle_matmul_bits(px, pw, ps, pb, y.ctypes.data_as(ctypes.c_void_p), M, N, K, bits):
+            raise ValueError("oracle rejected its arguments")
+        return y
+
+    def unpack_bits(self, wq, K: int, bits: int) -> np.ndarray:
+        wq, pw = _c(wq, np.uint32)
+        N = wq.shape[0]
+        q = np.empty((N, K), dtype=np.uint8)
+        if self.lib.w4a16_oracle_unpack_bits(pw, q.ctypes.data_as(ctypes.c_void_p), N, K, bits):
+            raise ValueError("oracle rejected its arguments")
+        return q
 
     def gate_up(self, x, wq, scales, biases) -> np.ndarray:
         """h [M, N2] BF16 bits = silu(gate) * up over interleaved gate/up rows (2 N2 rows)."""
@@ -180,14 +208,12 @@ def gate_up(x, wq, scales, biases):
     return default().gate_up(x, wq, scales, biases)
 
 
-def interleave_gate_up(gate, up):
-    """Row-interleave two [N2, ...] arrays (a packed layer's wq, scales or biases) in blocks
-    of 8: gate rows 8 b .. 8 b + 7, then up rows 8 b .. 8 b + 7 (a layout, no arithmetic)."""
-    gate, up = np.asarray(gate), np.asarray(up)
-    if gate.shape != up.shape or gate.shape[0] % 8:
-        raise ValueError("gate and up need the same shape and a row count divisible by 8")
-    n2 = gate.shape[0]
-    return np.stack([gate.reshape(n2 // 8, 8, -1), up.reshape(n2 // 8, 8, -1)], axis=1).reshape(2 * n2, -1)
+def matmul_bits(x, wq, scales, biases, bits):
+    return default().matmul_bits(x, wq, scales, biases, bits)
+
+
+def unpack_bits(wq, K, bits):
+    return default().unpack_bits(wq, K, bits)
 
 
 def unpack(wq, K):

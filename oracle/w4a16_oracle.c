@@ -28,6 +28,13 @@
  * / 15, bias = min, q = round and clamp to 0..15, eight codes per uint32 low
  * nibble first); the steps are spelled out above the function.
  *
+ * The same layer with 2- or 8-bit codes (w4a16_oracle_matmul_bits; the
+ * "Route affine qmv_wide by bit-width and batch size" PR routes the affine
+ * format by its bit width b): 32 / b codes per uint32, the lowest code in the
+ * lowest bits, so step 1 reads
+ *   q[n,k] = (wq[n*(K*b/32) + k/(32/b)] >> (b*(k%(32/b)))) & (2^b - 1)
+ * and steps 2-4 are unchanged.
+ *
  * BF16 values are passed as uint16_t bit patterns.
  */
 #include <math.h>
@@ -153,6 +160,61 @@ int w4a16_oracle_gate_up(const uint16_t *x, const uint32_t *wq, const uint16_t *
             const double uv = (double)dot_fp32(x, wq, s, b, K, m, up_row);
             h[m * N2 + j] = f32_to_bf16_rne((float)(silu(gv) * uv));
         }
+    return 0;
+}
+
+/*
+ * b-bit codes (b = 2, 4 or 8): step 1 with 32 / b codes per word, then steps 2-4 exactly
+ * as dot_fp32 takes them.
+ */
+static unsigned unpack_code_bits(const uint32_t *wq, int64_t K, int64_t n, int64_t k, int bits)
+{
+    const int64_t per_word = 32 / bits;
+    const uint32_t word = wq[n * (K / per_word) + k / per_word];
+    return (unsigned)((word >> (bits * (k % per_word))) & ((1u << bits) - 1u));
+}
+
+static float dot_fp32_bits(const uint16_t *x, const uint32_t *wq, const uint16_t *s,
+                           const uint16_t *b, int64_t K, int64_t m, int64_t n, int bits)
+{
+    const int64_t G = K / 128;
+    float acc = 0.0f;
+    for (int64_t k = 0; k < K; ++k) {
+        const float sc = bf16_to_f32(s[n * G + k / 128]);
+        const float bi = bf16_to_f32(b[n * G + k / 128]);
+        const float q = (float)unpack_code_bits(wq, K, n, k, bits);
+        const float sq = sc * q;
+        const float w = sq + bi;
+        const float xv = bf16_to_f32(x[m * K + k]);
+        const float p = xv * w;
+        acc = acc + p;
+    }
+    return acc;
+}
+
+/* y[M,N] bf16 bits = x[M,K] . dequant(wq)^T with b-bit codes; status 1 also for b not 2, 4, 8. */
+int w4a16_oracle_matmul_bits(const uint16_t *x, const uint32_t *wq, const uint16_t *s,
+                             const uint16_t *b, uint16_t *y, int64_t M, int64_t N,
+                             int64_t K, int bits)
+{
+    if ((bits != 2 && bits != 4 && bits != 8) || check(x, wq, s, b, y, M, N, K))
+        return 1;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t n = 0; n < N; ++n)
+            y[m * N + n] = f32_to_bf16_rne(dot_fp32_bits(x, wq, s, b, K, m, n, bits));
+    return 0;
+}
+
+/* Step 1 alone for b-bit codes: q[N,K] as bytes. */
+int w4a16_oracle_unpack_bits(const uint32_t *wq, uint8_t *q, int64_t N, int64_t K, int bits)
+{
+    if ((bits != 2 && bits != 4 && bits != 8) || N < 0 || K < 0 || K % (32 / bits) != 0 ||
+        (N > 0 && K > 0 && (!wq || !q)))
+        return 1;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            q[n * K + k] = (uint8_t)unpack_code_bits(wq, K, n, k, bits);
     return 0;
 }
 

@@ -345,9 +345,8 @@ def _gate_up_problem(gvals, uvals, K=128):
         return synth.pack_nibbles(q), synth.bf16_bits(np.ones((n2, K // 128), np.float32)), synth.bf16_bits(bias)
     gq, gs, gb = rows(gvals)
     uq, us, ub = rows(uvals)
-    from oracle import interleave_gate_up
     x = synth.bf16_bits(np.ones((1, K), np.float32))
-    return x, interleave_gate_up(gq, uq), interleave_gate_up(gs, us), interleave_gate_up(gb, ub)
+    return x, synth.interleave_gate_up(gq, uq), synth.interleave_gate_up(gs, us), synth.interleave_gate_up(gb, ub)
 
 
 def pin_gate_up_closed_forms(orc):
@@ -390,6 +389,111 @@ def pin_gate_up_odd_part(orc):
         assert abs(hp - hn - v) <= tol, (v, float(hp), float(hn))
 
 
+# ---------------------------------------------------------------- other bit widths
+# The affine format with b-bit codes: 32 / b codes per uint32, the lowest code in the
+# lowest bits; dequantisation and accumulation as for 4 bits.
+
+def pin_bits_unpack_hand_words(orc):
+    """Hand-built words: 0xE4 holds the 2-bit codes 0, 1, 2, 3 (low first), 0x1B holds
+    3, 2, 1, 0; 0x03020100 holds the bytes 0, 1, 2, 3; rows are words apart."""
+    wq2 = np.array([[0xE4E4E4E4, 0x0000001B], [0xFFFFFFFF, 0x00000000]], np.uint32)
+    want2 = np.array([[0, 1, 2, 3] * 4 + [3, 2, 1, 0] + [0] * 12, [3] * 16 + [0] * 16], np.uint8)
+    assert np.array_equal(orc.unpack_bits(wq2, 32, 2), want2)
+    wq8 = np.array([[0x03020100, 0xFF80017F], [0x00000010, 0x20000000]], np.uint32)
+    want8 = np.array([[0, 1, 2, 3, 0x7F, 0x01, 0x80, 0xFF], [0x10, 0, 0, 0, 0, 0, 0, 0x20]], np.uint8)
+    assert np.array_equal(orc.unpack_bits(wq8, 8, 8), want8)
+    # four bits read the nibble layout of the 4-bit format
+    assert np.array_equal(orc.unpack_bits(np.array([[0x76543210]], np.uint32), 8, 4), [[0, 1, 2, 3, 4, 5, 6, 7]])
+
+
+def pin_bits_onehot_reads_codes(orc):
+    """x = e_k, scale 1, bias 0: y[n] is the code of (n, k), for every k of two groups."""
+    for bits in (2, 8):
+        N, K = 3, 256
+        top = (1 << bits) - 1
+        q = (np.arange(N * K).reshape(N, K) * 37 + 11) % (top + 1)
+        wq = synth.pack_codes(q.astype(np.uint8), bits)
+        s = synth.bf16_bits(np.ones((N, 2), np.float32))
+        b = np.zeros((N, 2), np.uint16)
+        x = synth.bf16_bits(np.eye(K, dtype=np.float32))
+        y = synth.bf16_to_f32(orc.matmul_bits(x, wq, s, b, bits))
+        assert np.array_equal(y, q.T.astype(np.float32)), bits
+
+
+def pin_bits_integer_exact(orc):
+    """Integer inputs whose FP32 sums are exact: the output is the int64 result rounded once."""
+    for bits, shapes in ((2, ((5, 24, 384), (1, 8, 1024), (3, 17, 128))), (8, ((5, 24, 256), (2, 9, 128)))):
+        for (M, N, K) in shapes:
+            p = synth.make_integer_problem_bits(M, N, K, bits)
+            G = K // 128
+            w = (p["si"][:, :, None] * p["qi"].reshape(N, G, 128) + p["bi"][:, :, None]).reshape(N, K)
+            expect = p["xi"] @ w.T
+            assert np.abs(expect).max() < 2 ** 24
+            y = orc.matmul_bits(p["x"], p["wq"], p["scales"], p["biases"], bits)
+            assert np.array_equal(y, synth.bf16_bits(expect.astype(np.float32))), (bits, M, N, K)
+
+
+def pin_bits_rational_brute_force(orc):
+    """Tiny random problems of both widths against exact rationals: the BF16 output within
+    one BF16 ulp plus the FP32 recursive-summation bound of the exact value."""
+    from tolerance import ulp_bf16
+    u = Fraction(1, 1 << 24)
+    for (bits, M, N, K, seed) in ((2, 2, 3, 256, 4), (8, 2, 3, 256, 5), (8, 1, 2, 128, 6)):
+        p = synth.make_problem_bits(M, N, K, bits, seed=seed, outliers=True)
+        y = orc.matmul_bits(p["x"], p["wq"], p["scales"], p["biases"], bits)
+        xf = [[_bits_to_fraction(int(v)) for v in row] for row in p["x"]]
+        sf = [[_bits_to_fraction(int(v)) for v in row] for row in p["scales"]]
+        bf = [[_bits_to_fraction(int(v)) for v in row] for row in p["biases"]]
+        per = 32 // bits
+        for n in range(N):
+            w = [sf[n][k // 128] * ((int(p["wq"][n, k // per]) >> (bits * (k % per))) & ((1 << bits) - 1))
+                 + bf[n][k // 128] for k in range(K)]
+            for m in range(M):
+                terms = [xf[m][k] * w[k] for k in range(K)]
+                exact = sum(terms, Fraction(0))
+                slack = float((K + 2) * u * sum(abs(t) for t in terms))
+                ex = float(exact)
+                yv = float(synth.bf16_to_f32(y[m:m + 1, n])[0])
+                assert abs(yv - ex) <= float(ulp_bf16(np.array([ex]))[0]) + slack, (bits, m, n, yv, ex)
+
+
+def pin_bits_fp32_sequential_sum(orc):
+    """Every code 1, scale 1, bias 0, x = (1, 2^-24 x 126, -1): in FP32 taken in ascending k
+    each 2^-24 meets 1.0 at a tie and is lost (ties to even), so the sum is exactly 0; the
+    exact sum (or one in FP64, or one taken from the top) is 126 x 2^-24."""
+    K = 128
+    x = np.array([[1.0] + [2.0 ** -24] * 126 + [-1.0]], np.float32)
+    s = synth.bf16_bits(np.ones((1, 1), np.float32))
+    b = np.zeros((1, 1), np.uint16)
+    for bits in (2, 8):
+        wq = synth.pack_codes(np.ones((1, K), np.uint8), bits)
+        y = orc.matmul_bits(synth.bf16_bits(x), wq, s, b, bits)
+        assert int(y[0, 0]) == 0x0000, (bits, hex(int(y[0, 0])))
+
+
+def pin_bits_four_is_the_w4_layer(orc):
+    """bits = 4 is the 4-bit layer itself (pinned above) on the same words."""
+    p = synth.make_problem(3, 40, 384, seed=9)
+    assert np.array_equal(orc.matmul_bits(p["x"], p["wq"], p["scales"], p["biases"], 4),
+                          orc.matmul(p["x"], p["wq"], p["scales"], p["biases"]))
+
+
+def pin_bits_rejects_bad_arguments(orc):
+    x = np.zeros((1, 128), np.uint16)
+    s = np.zeros((1, 1), np.uint16)
+    for bits, words in ((3, 12), (16, 64), (1, 4)):
+        try:
+            orc.matmul_bits(x, np.zeros((1, words), np.uint32), s, s, bits)
+        except ValueError:
+            continue
+        raise AssertionError(f"bits={bits} was accepted")
+    try:
+        orc.matmul_bits(np.zeros((1, 136), np.uint16), np.zeros((1, 34), np.uint32), s, s, 8)
+    except ValueError:
+        return
+    raise AssertionError("K % 128 != 0 was accepted")
+
+
 ALL_PINS = (
     pin_unpack_hand_words,
     pin_onehot_reads_codes,
@@ -410,6 +514,13 @@ ALL_PINS = (
     pin_gate_up_closed_forms,
     pin_gate_up_interleave,
     pin_gate_up_odd_part,
+    pin_bits_unpack_hand_words,
+    pin_bits_onehot_reads_codes,
+    pin_bits_integer_exact,
+    pin_bits_fp32_sequential_sum,
+    pin_bits_rational_brute_force,
+    pin_bits_four_is_the_w4_layer,
+    pin_bits_rejects_bad_arguments,
 )
 
 

@@ -45,6 +45,24 @@ MUTANTS = {
     "up_row_is_gate_row": ("const int64_t up_row = gate_row + 8;", "const int64_t up_row = gate_row;"),
     "silu_sign": ("return g / (1.0 + exp(-g));", "return g / (1.0 + exp(g));"),
     "silu_dropped": ("f32_to_bf16_rne((float)(silu(gv) * uv))", "f32_to_bf16_rne((float)(gv * uv))"),
+    # other bit widths
+    "bits_code_order_reversed": ("(word >> (bits * (k % per_word)))", "(word >> (bits * (per_word - 1 - k % per_word)))"),
+    "bits_mask_one_bit_short": ("((1u << bits) - 1u)", "((1u << (bits - 1)) - 1u)"),
+    "bits_word_stride_of_4_bits": ("wq[n * (K / per_word) + k / per_word]", "wq[n * (K / 8) + k / per_word]"),
+    "bits_eight_per_word": ("const int64_t per_word = 32 / bits;", "const int64_t per_word = 8;"),
+    "bits_ignored": ("(float)unpack_code_bits(wq, K, n, k, bits)", "(float)unpack_code_bits(wq, K, n, k, 4)"),
+}
+
+# Mistakes planted only in the b-bit dot product (its text repeats the 4-bit one's): the
+# first occurrence after the anchor is replaced.
+BITS_ANCHOR = "static float dot_fp32_bits("
+BITS_MUTANTS = {
+    "bits_bias_dropped": ("const float w = sq + bi;", "const float w = sq;"),
+    "bits_scale_dropped": ("const float sq = sc * q;", "const float sq = q;"),
+    "bits_scale_group_index": ("bf16_to_f32(s[n * G + k / 128])", "bf16_to_f32(s[n * G + (k / 128) % 1])"),
+    "bits_x_index": ("x[m * K + k]", "x[m * K + (k ^ 1)]"),
+    "bits_fp64_accumulator": ("float acc = 0.0f;", "double acc = 0.0;"),
+    "bits_k_descending": ("for (int64_t k = 0; k < K; ++k) {", "for (int64_t k = K - 1; k >= 0; --k) {"),
 }
 
 
@@ -80,6 +98,17 @@ def test_mutant_is_caught(tmp_path, name):
     lib = _build(tmp_path, name, text.replace(old, new))
     rc, out = _run_pins(lib)
     assert rc != 0, f"{name} survived every pin: {out}"
+
+
+@pytest.mark.parametrize("name", sorted(BITS_MUTANTS))
+def test_bits_mutant_is_caught(tmp_path, name):
+    old, new = BITS_MUTANTS[name]
+    text = open(oracle.SOURCE).read()
+    a = text.index(BITS_ANCHOR)
+    i = text.index(old, a)
+    lib = _build(tmp_path, name, text[:i] + new + text[i + len(old):])
+    rc, out = _run_pins(lib)
+    assert rc != 0 and "pin_bits" in out, f"{name} survived the b-bit pins: {out}"
 
 
 def test_fused_multiply_add_is_caught(tmp_path):

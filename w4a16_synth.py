@@ -231,3 +231,69 @@ def interleave_gate_up(gate, up):
         raise ValueError("gate and up need the same shape and a row count divisible by 8")
     n2 = gate.shape[0]
     return np.stack([gate.reshape(n2 // 8, 8, -1), up.reshape(n2 // 8, 8, -1)], axis=1).reshape(2 * n2, -1)
+
+
+# ---------------------------------------------------------------- other bit widths
+# The same affine format with b-bit codes (b in {2, 4, 8}): 32 / b codes per uint32, low first,
+# scale = (max - min) / (2^b - 1), q clamped to 0 .. 2^b - 1; wq is [N, K * b / 32].
+
+def pack_codes(q: np.ndarray, bits: int) -> np.ndarray:
+    """uint8 codes [N, K] in 0 .. 2^bits - 1 -> uint32 words [N, K * bits / 32], low first."""
+    q = np.asarray(q)
+    N, K = q.shape
+    per = 32 // bits
+    if bits not in (2, 4, 8) or K % per:
+        raise ValueError("bits must be 2, 4 or 8 and K a multiple of 32 / bits")
+    if q.min(initial=0) < 0 or q.max(initial=0) > (1 << bits) - 1:
+        raise ValueError("codes out of range")
+    q = q.astype(np.uint32).reshape(N, K // per, per)
+    shifts = (bits * np.arange(per, dtype=np.uint32))[None, None, :]
+    return np.bitwise_or.reduce(q << shifts, axis=2).astype(np.uint32)
+
+
+def quantize_affine_g128(W: np.ndarray, bits: int):
+    """The min/max recipe of quantize_w4_g128 for b-bit codes (2^b - 1 steps per group)."""
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    if K % GROUP:
+        raise ValueError("K must be a multiple of 128")
+    top = (1 << bits) - 1
+    Wg = W.reshape(N, K // GROUP, GROUP)
+    mn = Wg.min(axis=2)
+    mx = Wg.max(axis=2)
+    s_bits = bf16_bits((mx - mn) / np.float32(top))
+    b_bits = bf16_bits(mn)
+    s = bf16_to_f32(s_bits)[..., None]
+    b = bf16_to_f32(b_bits)[..., None]
+    safe = np.where(s == 0, np.float32(1), s)
+    q = np.rint((Wg - b) / safe)
+    q = np.where(s == 0, 0, q)
+    q = np.clip(q, 0, top).astype(np.uint8).reshape(N, K)
+    return pack_codes(q, bits), s_bits, b_bits
+
+
+def make_problem_bits(M: int, N: int, K: int, bits: int, seed: int = 0, outliers: bool = False) -> dict:
+    """make_problem with b-bit codes (its own stream per shape and bit width)."""
+    rng = np.random.default_rng([seed, M, N, K, bits])
+    x = make_x(rng, M, K, outliers=outliers)
+    W = rng.standard_normal((N, K), dtype=np.float32) * np.float32(0.02)
+    wq, s, b = quantize_affine_g128(W, bits)
+    return {"x": x, "wq": wq, "scales": s, "biases": b, "M": M, "N": N, "K": K, "bits": bits}
+
+
+def make_integer_problem_bits(M: int, N: int, K: int, bits: int, seed: int = 0) -> dict:
+    """Integer-valued inputs with b-bit codes whose FP32 sums are exact (see make_integer_problem):
+    x in {-4..4}, scale in {1, 2}, bias in {-8..0}, codes in 0 .. 2^bits - 1, K <= 1024 for
+    bits <= 4 and K <= 256 for 8 bits (|partial sums| < 2^24)."""
+    rng = np.random.default_rng([seed + 7919, M, N, K, bits])
+    G = K // GROUP
+    xi = rng.integers(-4, 5, size=(M, K)).astype(np.int64)
+    qi = rng.integers(0, 1 << bits, size=(N, K)).astype(np.uint8)
+    si = rng.integers(1, 3, size=(N, G)).astype(np.int64)
+    bi = rng.integers(-8, 1, size=(N, G)).astype(np.int64)
+    return {
+        "x": bf16_bits(xi.astype(np.float32)), "wq": pack_codes(qi, bits),
+        "scales": bf16_bits(si.astype(np.float32)), "biases": bf16_bits(bi.astype(np.float32)),
+        "M": M, "N": N, "K": K, "bits": bits,
+        "xi": xi, "qi": qi.astype(np.int64), "si": si, "bi": bi,
+    }
