@@ -470,6 +470,9 @@ def run_ours(args, world, rank, local):
         gate_up = gate_up_section(device, stream, pk)
     if not args.no_prefill and rank == 0:
         skinny = skinny_section(device, stream, pk, weights_cache)
+    nbits = None
+    if not args.no_quantize and rank == 0:
+        nbits = bits_section(device, stream, pk)
 
     if rank == 0:
         line = {
@@ -504,6 +507,8 @@ def run_ours(args, world, rank, local):
             line["gate_up"] = gate_up
         if skinny is not None:
             line["skinny"] = skinny
+        if nbits is not None:
+            line["bits"] = nbits
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
@@ -688,6 +693,55 @@ def gate_up_section(device, stream, pk):
                              "fused fraction of measured HBM"]}
 
 
+def bits_algo_bytes(M, N, K, bits):
+    """Bytes a b-bit layer call must move at least: codes, scales and biases once, x and y once."""
+    return N * K * bits // 8 + 4 * N * (K // 128) + 2 * M * K + 2 * M * N
+
+
+def bits_section(device, stream, pk):
+    """Decode (M in {1, 8}) over the seven Qwen3-4B projections with 2-, 4- and 8-bit codes
+    through w4a16_matmul_bits (4 bits: the 4-bit layer's own path).  Codes are random words and
+    scales / biases small random BF16 values generated on the device: the timing depends on
+    the bytes, not on the values."""
+    import torch
+    import decode_w4a16_g128_b200 as w4
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    g = torch.Generator(device=device).manual_seed(2024)
+    rows, summary = [], {}
+    for bits in (2, 4, 8):
+        for M in (1, 8):
+            tot_us, tot_b = 0.0, 0
+            for (name, K, N) in synth.QWEN3_4B_PROJECTIONS:
+                G = K // 128
+                base = (torch.randn((M, K), generator=g, device=device).to(torch.bfloat16),
+                        torch.randint(-2 ** 31, 2 ** 31 - 1, (N, K * bits // 32), generator=g, device=device,
+                                      dtype=torch.int32),
+                        (0.002 + 0.001 * torch.rand((N, G), generator=g, device=device)).to(torch.bfloat16),
+                        (-0.03 - 0.01 * torch.rand((N, G), generator=g, device=device)).to(torch.bfloat16))
+                b = bits_algo_bytes(M, N, K, bits)
+                n_copies = int(max(2, min(16, math.ceil(2.2 * l2 / b))))
+
+                def make_copy(i, base=base, M=M, N=N):
+                    t = base if i == 0 else tuple(a.clone() for a in base)
+                    return t + (torch.empty((M, N), dtype=torch.bfloat16, device=device),)
+
+                def launch(c, bits=bits):
+                    w4.w4a16_matmul_bits(c[0], c[1], c[2], c[3], bits, y=c[4])
+
+                us = time_calls(make_copy, launch, n_copies, 16, stream)
+                del base
+                rows.append([bits, M, name, N, K, round(us, 3), round(b / us / 1e3, 1)])
+                tot_us += us
+                tot_b += b
+            summary[f"{bits}bit_m{M}"] = {"us": round(tot_us, 3), "gbs": round(tot_b / tot_us / 1e3, 1),
+                                          "frac": round(tot_b / tot_us / 1e3 / pk["hbm_gbs"], 4)}
+    torch.cuda.empty_cache()
+    return {"workload": "decode M in {1, 8}, seven Qwen3-4B projections, 2-, 4- and 8-bit affine codes, g128",
+            "kernel": "w4a16::nb::nbit_kernel<2|8> (4 bits: the 4-bit layer's decode path)", "bound": "hbm",
+            "peak": pk["hbm_gbs"], "summary": summary, "calls": rows,
+            "calls_fields": ["bits", "M", "projection", "N", "K", "us", "GB/s"]}
+
+
 def skinny_section(device, stream, pk, weights_cache):
     """8 < M <= 32: slices of the row-block matvec against the GEMM, per Qwen3-4B projection
     (the measured crossover behind the automatic choice)."""
@@ -725,7 +779,8 @@ def skinny_section(device, stream, pk, weights_cache):
 
 def profile_case(args, device, stream):
     """Three eager calls of one problem (for an ncu capture of one kernel): 'M,N,K' (the layer),
-    'quant:N,K,f32|bf16' (the quantiser) or 'gateup:M,N2,K' (the fused gate/up projection)."""
+    'quant:N,K,f32|bf16' (the quantiser), 'gateup:M,N2,K' (the fused gate/up projection) or
+    'bits:b,M,N,K' (the layer with b-bit codes)."""
     import torch
     import decode_w4a16_g128_b200 as w4
     if args.case.startswith("quant:"):
@@ -739,6 +794,19 @@ def profile_case(args, device, stream):
             for _ in range(3):
                 w4.w4a16_quantize(W)
         torch.cuda.synchronize()
+        return 0
+    if args.case.startswith("bits:"):
+        bits, M, N, K = (int(v) for v in args.case[len("bits:"):].split(","))
+        prob = synth.make_problem_bits(M, N, K, bits)
+        d = [torch.from_numpy(prob[k].view(np.int16 if prob[k].dtype == np.uint16 else np.int32)).to(device)
+             for k in ("x", "wq", "scales", "biases")]
+        with torch.cuda.stream(stream):
+            for _ in range(3):
+                w4.w4a16_matmul_bits(d[0].view(torch.bfloat16), d[1], d[2].view(torch.bfloat16),
+                                     d[3].view(torch.bfloat16), bits)
+        torch.cuda.synchronize()
+        if w4.w4a16_device_status(stream) != w4.OK:
+            raise RuntimeError("device status not ok")
         return 0
     if args.case.startswith("gateup:"):
         M, N2, K = (int(v) for v in args.case[len("gateup:"):].split(","))
@@ -822,7 +890,8 @@ def main():
                     help="also time every decode call on its own and write the table to PATH (JSON)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-prefill", action="store_true", help="skip the M > 8 measurements")
-    ap.add_argument("--no-quantize", action="store_true", help="skip the quantiser measurement")
+    ap.add_argument("--no-quantize", action="store_true",
+                    help="skip the quantiser, fused gate/up and 2- / 8-bit measurements")
     ap.add_argument("--cpu-seconds", type=float, default=10.0, help="time bound of the CPU baseline sample")
     ap.add_argument("--case", default="", help="profile mode: one problem 'M,N,K' (three eager calls)")
     ap.add_argument("--ref-fraction", type=float, default=0.125,

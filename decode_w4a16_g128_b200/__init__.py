@@ -83,9 +83,10 @@ def _load() -> ctypes.CDLL:
     lib.w4a16_matvec_noalloc.argtypes = [p, p, p, p, p, i64, i64, i64, p]
     lib.w4a16_quantize.argtypes = [p, ctypes.c_int32, p, p, p, i64, i64, p]
     lib.w4a16_gate_up.argtypes = [p, p, p, p, p, i64, i64, i64, p]
+    lib.w4a16_matmul_bits.argtypes = [p, p, p, p, p, i64, i64, i64, ctypes.c_int32, p]
     for name in ("w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan",
                  "w4a16_device_status", "w4a16_last_cuda_error", "w4a16_version", "w4a16_matvec_noalloc",
-                 "w4a16_quantize", "w4a16_gate_up"):
+                 "w4a16_quantize", "w4a16_gate_up", "w4a16_matmul_bits"):
         getattr(lib, name).restype = i32
     return lib
 
@@ -222,6 +223,34 @@ def w4a16_gate_up(x, wq, scales, biases, h=None, stream=None):
     return h
 
 
+def w4a16_matmul_bits(x, wq, scales, biases, bits: int, y=None, stream=None):
+    """y = x . dequant(wq)^T with b-bit codes (b = 2, 4 or 8): wq int32/uint32 [N, K b / 32], 32 / b
+    codes per word, the lowest code in the lowest bits.  2 and 8 bits: M <= 32."""
+    import torch
+    if bits not in (2, 4, 8):
+        raise W4A16Error(ERR_UNSUPPORTED, "w4a16_matmul_bits")
+    if x.dtype != torch.bfloat16 or scales.dtype != torch.bfloat16 or biases.dtype != torch.bfloat16:
+        raise TypeError("x, scales and biases must be bfloat16")
+    if wq.dtype not in (torch.int32, torch.uint32):
+        raise TypeError("wq must be int32 or uint32 (packed codes)")
+    for name, t in (("x", x), ("wq", wq), ("scales", scales), ("biases", biases)):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CUDA tensor")
+    M, K = x.shape
+    N = wq.shape[0]
+    if tuple(wq.shape) != (N, K * bits // 32) or tuple(scales.shape) != (N, K // 128) or \
+            tuple(biases.shape) != (N, K // 128):
+        raise ValueError(f"shape mismatch: x {tuple(x.shape)}, wq {tuple(wq.shape)}, "
+                         f"scales {tuple(scales.shape)}, biases {tuple(biases.shape)} for {bits}-bit codes")
+    if y is None:
+        y = torch.empty((M, N), dtype=torch.bfloat16, device=x.device)
+    elif tuple(y.shape) != (M, N) or y.dtype != torch.bfloat16 or not y.is_cuda or not y.is_contiguous():
+        raise ValueError("y must be a contiguous bfloat16 CUDA tensor [M, N]")
+    _check(lib.w4a16_matmul_bits(_ptr(x), _ptr(wq), _ptr(scales), _ptr(biases), _ptr(y), M, N, K, int(bits),
+                                 _stream_handle(stream)), "w4a16_matmul_bits")
+    return y
+
+
 def w4a16_quantize(w, wq=None, scales=None, biases=None, stream=None):
     """Quantise weights W [N, K] (float32 or bfloat16, CUDA, contiguous) on the GPU into the
     packed format: returns (wq int32 [N, K/8], scales bf16 [N, K/128], biases bf16 [N, K/128])."""
@@ -277,7 +306,7 @@ def w4a16_streamk_owner(units: int, workers: int, u: int) -> int:
 __all__ = [
     "w4a16_matmul", "w4a16_matmul_ex", "w4a16_matmul_last_rows", "w4a16_plan", "w4a16_device_status",
     "w4a16_release", "w4a16_version", "w4a16_streamk_owner", "w4a16_matvec_noalloc", "w4a16_quantize",
-    "w4a16_gate_up", "interleave_gate_up",
+    "w4a16_gate_up", "interleave_gate_up", "w4a16_matmul_bits",
     "status_string", "W4A16Error", "Options",
     "PlanInfo", "make_options", "lib", "LIBRARY_PATH",
 ]

@@ -19,6 +19,7 @@
 
 #include "gemm.cuh"
 #include "matvec.cuh"
+#include "nbit.cuh"
 #include "quant.cuh"
 #include "rows.cuh"
 
@@ -795,6 +796,75 @@ int matmul_impl(const Problem &p, void *stream, const w4a16_options *opt) {
     return launch_gemm(d, ws, p, pl, stream, pdl, pdl && static_weights);
 }
 
+// ------------------------------------------------------------------ 2- and 8-bit codes
+
+constexpr int64_t kBitsMaxM = 32;   // slices of 8 x rows, as the 4-bit row-block path
+
+template <int BITS>
+int launch_nbit(const Problem &p, void *stream) {
+    nb::Params kp;
+    kp.x = static_cast<const uint16_t *>(p.x);
+    kp.wq = p.wq;
+    kp.scales = static_cast<const uint16_t *>(p.scales);
+    kp.biases = static_cast<const uint16_t *>(p.biases);
+    kp.y = static_cast<uint16_t *>(p.y);
+    kp.M = static_cast<int>(p.M);
+    kp.N = static_cast<int>(p.N);
+    kp.K = static_cast<int>(p.K);
+    kp.G = static_cast<int>(p.K / 128);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>((p.N + nb::rows_per_cta<BITS>() - 1) / nb::rows_per_cta<BITS>()), 1, 1);
+    cfg.blockDim = dim3(nb::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = static_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, nb::nbit_kernel<BITS>, kp);
+    return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+}
+
+int matmul_bits_impl(const Problem &p, int bits, void *stream) {
+    if (bits == 4) return matmul_impl(p, stream, nullptr);
+    if (p.M < 0 || p.N < 0 || p.K < 0) return W4A16_ERR_INVALID_ARG;
+    if (bits != 2 && bits != 8) return W4A16_ERR_UNSUPPORTED;
+    if (p.K % 128 != 0 || p.M > kBitsMaxM || p.N >= (int64_t(1) << 31) || p.K >= (int64_t(1) << 31))
+        return W4A16_ERR_UNSUPPORTED;
+    if (p.M == 0 || p.N == 0) return W4A16_OK;
+    if (!p.y) return W4A16_ERR_INVALID_ARG;
+    if (!aligned16(p.y)) return W4A16_ERR_MISALIGNED;
+    if (p.K > 0) {
+        if (!p.x || !p.wq || !p.scales || !p.biases) return W4A16_ERR_INVALID_ARG;
+        if (!aligned16(p.x) || !aligned16(p.wq) || !aligned16(p.scales) || !aligned16(p.biases))
+            return W4A16_ERR_MISALIGNED;
+        const size_t ny = size_t(p.M) * p.N * 2;
+        if (overlaps(p.y, ny, p.x, size_t(p.M) * p.K * 2) || overlaps(p.y, ny, p.wq, size_t(p.N) * p.K * bits / 8) ||
+            overlaps(p.y, ny, p.scales, size_t(p.N) * (p.K / 128) * 2) ||
+            overlaps(p.y, ny, p.biases, size_t(p.N) * (p.K / 128) * 2))
+            return W4A16_ERR_INVALID_ARG;
+    }
+    int dev = 0;
+    int rc = current_device(&dev);
+    if (rc) return rc;
+    std::lock_guard<std::mutex> lock(g_mu);
+    DeviceInfo *d = nullptr;
+    rc = device_setup(dev, &d);
+    if (rc) return rc;
+    if (p.K == 0) {   // an empty sum: every output is +0
+        cudaError_t e = cudaMemsetAsync(p.y, 0, size_t(p.M) * p.N * 2, static_cast<cudaStream_t>(stream));
+        return e == cudaSuccess ? W4A16_OK : cuda_fail(e);
+    }
+    for (int64_t m0 = 0; m0 < p.M; m0 += nb::kMaxM) {
+        const Problem sub{static_cast<const uint16_t *>(p.x) + m0 * p.K, p.wq, p.scales, p.biases,
+                          static_cast<uint16_t *>(p.y) + m0 * p.N, std::min<int64_t>(nb::kMaxM, p.M - m0), p.N, p.K};
+        rc = bits == 2 ? launch_nbit<2>(sub, stream) : launch_nbit<8>(sub, stream);
+        if (rc) return rc;
+    }
+    return W4A16_OK;
+}
+
 // ------------------------------------------------------------------ allocation-free matvec
 
 // Scratch of w4a16_matvec_noalloc: a region for the FP32 partials of up to
@@ -1023,6 +1093,11 @@ int w4a16_gate_up(const void *x, const uint32_t *wq, const void *scales, const v
         if (rc) return rc;
     }
     return W4A16_OK;
+}
+
+int w4a16_matmul_bits(const void *x, const uint32_t *wq, const void *scales, const void *biases, void *y,
+                      int64_t M, int64_t N, int64_t K, int32_t bits, void *stream) {
+    return matmul_bits_impl(Problem{x, wq, scales, biases, y, M, N, K}, bits, stream);
 }
 
 int w4a16_quantize(const void *w, int32_t w_dtype, uint32_t *wq, void *scales, void *biases, int64_t N, int64_t K,

@@ -287,6 +287,28 @@ enum w4a16_dtype {
 int w4a16_quantize(const void *w, int32_t w_dtype, uint32_t *wq, void *scales,
                    void *biases, int64_t N, int64_t K, void *stream);
 
+/*
+ * The same layer with 2- or 8-bit codes (the "Route affine qmv_wide by
+ * bit-width and batch size" PR routes the affine format by its bit width b):
+ *   y[m,n] = bf16_rne( sum_k x[m,k] * (scale[n,k/128] * q[n,k] + bias[n,k/128]) )
+ * with q[n,k] = (wq[n*(K*b/32) + k/(32/b)] >> (b*(k%(32/b)))) & (2^b - 1):
+ * 32 / b codes per uint32, the lowest code in the lowest bits.  x, scales,
+ * biases and y are as in w4a16_matmul; wq is [N, K*b/32] uint32.  FP32
+ * accumulation; the result is within one BF16 ulp (+ 1e-3 absolute) of the
+ * plain sequential FP32 definition, and does not depend on timing.
+ *
+ * bits = 4 is w4a16_matmul itself (every path, any M).  bits = 2 and 8 run a
+ * tensor-core matvec for decode: M <= 32 (in launches of 8 x rows; larger M
+ * gives W4A16_ERR_UNSUPPORTED), any N, K % 128 == 0.  Other bit widths give
+ * W4A16_ERR_UNSUPPORTED.  Size, alignment, overlap, K == 0 and stream rules
+ * are those of w4a16_matmul (wq spans N*K*b/8 bytes); every launch uses the
+ * programmatic-dependent-launch attribute and waits for the preceding kernel
+ * before its first read.
+ */
+int w4a16_matmul_bits(const void *x, const uint32_t *wq, const void *scales,
+                      const void *biases, void *y, int64_t M, int64_t N, int64_t K,
+                      int32_t bits, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

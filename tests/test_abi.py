@@ -281,3 +281,31 @@ def test_matvec_default_workers(N, K, expect):
     pl = w4.w4a16_plan(1, N, K, path=w4.PATH_MATVEC, sm_count=148)
     assert pl["path"] == w4.PATH_MATVEC and pl["grid_x"] == expect
     assert w4.w4a16_plan(1, N, K, sm_count=148, workers=17)["grid_x"] == min(17, pl["units"])
+
+
+def mmb(x, wq, s, b, y, M, N, K, bits):
+    return lib.w4a16_matmul_bits(P(x), P(wq), P(s), P(b), P(y), M, N, K, bits, P(0))
+
+
+def test_bits_argument_checks():
+    good = [A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x400000]
+    for bits in (2, 8):
+        assert mmb(*good, -1, 8, 128, bits) == w4.ERR_INVALID_ARG
+        assert mmb(*good, 1, 8, 136, bits) == w4.ERR_UNSUPPORTED
+        assert mmb(*good, 33, 8, 128, bits) == w4.ERR_UNSUPPORTED       # decode only: M <= 32
+        assert mmb(0, 0, 0, 0, 0, 0, 8, 128, bits) == w4.OK               # empty: no GPU needed
+        assert mmb(0, 0, 0, 0, 0, 4, 0, 128, bits) == w4.OK
+        for i in range(5):
+            args = list(good)
+            args[i] = 0
+            assert mmb(*args, 2, 8, 256, bits) == w4.ERR_INVALID_ARG
+            args = list(good)
+            args[i] += 8
+            assert mmb(*args, 2, 8, 256, bits) == w4.ERR_MISALIGNED
+    for bits in (0, 1, 3, 5, 16, 32, -4):
+        assert mmb(*good, 1, 8, 128, bits) == w4.ERR_UNSUPPORTED
+    # y inside the codes: 8-bit codes of 64 rows x 1024 take 64 KB, 2-bit ones 16 KB
+    assert mmb(A, A + 0x100000, A + 0x200000, A + 0x300000, A + 0x100000 + 0xC000, 1, 64, 1024, 8) == w4.ERR_INVALID_ARG
+    # bits = 4 is the 4-bit layer's own validation
+    assert mmb(*good, 1, 8, 136, 4) == w4.ERR_UNSUPPORTED
+    assert mmb(0, 0, 0, 0, 0, 0, 8, 128, 4) == w4.OK
