@@ -37,30 +37,3 @@ __device__ __forceinline__ float plain_output(const uint16_t *x_row, const uint3
 }
 
 }  // namespace w4a16
-
-namespace w4a16 {
-
-// The same for b-bit codes (b = 2 or 8): 32 / b codes per word, the lowest code in the lowest bits.
-template <int BITS>
-__device__ __forceinline__ float plain_output_bits(const uint16_t *x_row, const uint32_t *wq_row, const uint16_t *s_row,
-                                                const uint16_t *b_row, int G) {
-    constexpr int kPer = 32 / BITS;
-    constexpr uint32_t kMask = (1u << BITS) - 1u;
-    float acc = 0.f;
-    for (int g = 0; g < G; ++g) {
-        const float s = __uint_as_float(static_cast<uint32_t>(s_row[g]) << 16);
-        const float b = __uint_as_float(static_cast<uint32_t>(b_row[g]) << 16);
-        for (int j = 0; j < 4 * BITS; ++j) {
-            const uint32_t word = wq_row[g * 4 * BITS + j];
-            for (int i = 0; i < kPer; ++i) {
-                const float q = static_cast<float>((word >> (BITS * i)) & kMask);
-                const float w = __fadd_rn(__fmul_rn(s, q), b);
-                const float x = __uint_as_float(static_cast<uint32_t>(x_row[g * 128 + kPer * j + i]) << 16);
-                acc = __fadd_rn(acc, __fmul_rn(x, w));
-            }
-        }
-    }
-    return acc;
-}
-
-}  // namespace w4a16
